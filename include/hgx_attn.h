@@ -1,0 +1,185 @@
+/*
+ * hgx_attn.h -- C ABI of the hybrid-masked GQA attention core of unified text+pixel
+ * transformers, for NVIDIA B200 (sm_100a).
+ *
+ * One call computes, for a packed batch of mixed text+image token sequences,
+ *
+ *   q' = rope(rmsnorm(q) * wq),  k' = rope(rmsnorm(k) * wk)      (in place, bf16)
+ *   out[b, i, h] = sum_{j visible from i} softmax_j(q'[i,h] . k'[j,h/4] * scale) v[j,h/4]
+ *
+ * Sources (named by page title and section):
+ *  - Shapes (32 query heads over 8 KV heads, head_dim 128), "q/k RMSNorm", "3-axis
+ *    interleaved mRoPE [24,20,20] at theta 5e6", the sequence layout
+ *    [text ... <|boi|><|tms|>] + [target patches] + [reference patches] and its mask
+ *    (text causal, generation tokens see everything): "hidream-o1-p100a" model card,
+ *    "What this model is".
+ *  - Condition and text tokens causal, generation tokens attend to everything including
+ *    the condition tokens: "HiDream-O1-Image" summary (genai-atlas), "How it works".
+ *  - Generalized Causal Attention (text rows see all previous tokens; image rows see all
+ *    previous tokens plus their whole image segment): "HunyuanImage 3.0 Technical Report"
+ *    (paper-graph-ui summary), section 3.4, "The core rule"; bud-325 summary, "Key claims".
+ *  - RoPE pairing: the half-split layout [cos(n t0), cos(n t1), ..., sin(n t0), ...] of the
+ *    1D RoPE definition, same report, section 3.4, "Generalized 2D Rotary Position
+ *    Embedding (RoPE)": feature k is rotated together with feature k + head_dim/2.
+ *  - Rejecting bad requests before any device work: model card, "Serving (HTTP)"
+ *    (contract errors return without touching the card).
+ *
+ * Readings where the pages are silent: softmax scale 1/sqrt(head_dim); RMSNorm eps inside
+ * the square root, weight multiplies, one weight vector shared by all heads; RMSNorm
+ * before RoPE; query head h reads KV head h / (Hq / Hkv); "interleaved [24,20,20]" drives
+ * frequency k by axis h when k % 3 == 1 and k < 60, by axis w when k % 3 == 2 and k < 60,
+ * and by axis t otherwise.
+ *
+ * Data layout (all device tensors row-major, packed varlen: the tokens of all batch
+ * elements back to back, T = cu_seqlens[batch] tokens in total):
+ *   q    bf16 [T, 32, 128]  (token stride 8192 B)      -- overwritten with q'
+ *   k    bf16 [T, 8, 128]   (token stride 2048 B)      -- overwritten with k'
+ *   v    bf16 [T, 8, 128]                               -- read only
+ *   out  bf16 [T, 32, 128]                              -- written
+ *   pos  int32 [T, 3]  (t, h, w) position of each token -- read only
+ *   wq, wk bf16 [128]  RMSNorm weights                  -- read only
+ * Every device pointer must be non-null (when T > 0) and 16-byte aligned; out must not
+ * overlap q, k or v. V must be finite: the kernel multiplies masked probabilities (exact
+ * zeros) with key rows of the neighbouring batch element, and 0 * inf is NaN.
+ *
+ * Segments: for batch element b, segs[cu_segs[b] .. cu_segs[b+1]) describe its tokens in
+ * order. Each has a start local to the element, a length >= 1 and a kind. They must tile
+ * [0, L_b) exactly, L_b = cu_seqlens[b+1] - cu_seqlens[b]. An element with L_b == 0 has
+ * no segments. Visibility of key j from query i (both local):
+ *   HGX_SEG_CAUSAL           j <= i
+ *   HGX_SEG_FULL_SEQUENCE    every j < L_b
+ *   HGX_SEG_FULL_IN_SEGMENT  j <= i, or j inside i's own segment
+ * Under all three kinds the visible keys of a row form a prefix [0, lim(i)).
+ *
+ * Ownership and threading: the caller owns every tensor and the stream. The handle owns
+ * the planner's device scratch (per-row key limits, the work list, a device error word)
+ * and reuses it while the segment descriptor is unchanged. A handle serves one stream at a
+ * time and is not thread-safe; calls on one handle must not overlap on the GPU unless they
+ * share a stream. Device calls are asynchronous on `stream` (a cudaStream_t, NULL for the
+ * legacy default stream).
+ *
+ * Errors: every export returns hgx_status. Descriptor and pointer checks run on the host
+ * before any device work; on failure nothing is launched and hgx_attn_last_error() gives a
+ * message. CUDA launch failures return HGX_ERR_CUDA. Every wait inside the attention kernel
+ * is bounded in time; a wait that runs out sets a device error word and the kernel returns
+ * early. hgx_attn_sync_status() (called automatically in checked mode) synchronizes the
+ * stream and reports that as HGX_ERR_TIMEOUT.
+ */
+#ifndef HGX_ATTN_H
+#define HGX_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HGX_OK = 0,
+  HGX_ERR_INVALID_ARG = 1, /* malformed descriptor, null or misaligned pointer, bad size */
+  HGX_ERR_UNSUPPORTED = 2, /* valid request outside what this build implements (shapes) */
+  HGX_ERR_OOM = 3,         /* device or pinned host allocation for the planner failed */
+  HGX_ERR_CUDA = 4,        /* a CUDA runtime or driver call failed */
+  HGX_ERR_TIMEOUT = 5      /* a bounded device wait ran out (see hgx_attn_sync_status) */
+} hgx_status;
+
+typedef enum {
+  HGX_SEG_CAUSAL = 0,
+  HGX_SEG_FULL_SEQUENCE = 1,
+  HGX_SEG_FULL_IN_SEGMENT = 2
+} hgx_seg_kind;
+
+typedef enum { HGX_TILE_SKIP = 0, HGX_TILE_PARTIAL = 1, HGX_TILE_FULL = 2 } hgx_tile_class;
+
+typedef struct {
+  int32_t start; /* first token, local to the batch element */
+  int32_t len;   /* >= 1 */
+  int32_t kind;  /* hgx_seg_kind */
+} hgx_segment;
+
+typedef struct {
+  int32_t num_q_heads;      /* must be 32 */
+  int32_t num_kv_heads;     /* must be 8 */
+  int32_t head_dim;         /* must be 128 */
+  double rope_theta;        /* > 0; 5e6 in the model card */
+  int32_t mrope_section[3]; /* (t, h, w) frequency counts, sum head_dim / 2; {24, 20, 20} */
+  float rms_eps;            /* >= 0; 1e-6 */
+  float softmax_scale;      /* > 0, or 0 for 1 / sqrt(head_dim) */
+} hgx_attn_config;
+
+typedef struct hgx_attn_handle hgx_attn_handle;
+
+/* Fills *cfg with the model card's constants (32/8/128, theta 5e6, [24,20,20], eps 1e-6,
+ * scale 0 = 1/sqrt(128)). */
+void hgx_attn_default_config(hgx_attn_config* cfg);
+
+/* Validates *cfg and creates a handle. No device memory is allocated until the first
+ * device call. Errors: INVALID_ARG (null, bad values), UNSUPPORTED (other shapes), OOM. */
+hgx_status hgx_attn_create(const hgx_attn_config* cfg, hgx_attn_handle** out);
+
+/* Frees the handle and its device scratch. Waits for nothing: the caller must make sure
+ * no call on the handle is still running on the GPU. NULL is ignored. */
+void hgx_attn_destroy(hgx_attn_handle* h);
+
+/* Message of the last failed call on this handle ("" if none). Valid until the next call. */
+const char* hgx_attn_last_error(const hgx_attn_handle* h);
+
+/* The whole path: prologue (RMSNorm + mRoPE of q and k, in place), then masked GQA
+ * attention into out. cu_seqlens_host int32 [batch+1] with cu_seqlens_host[0] == 0, and
+ * segs_host / cu_segs_host (int32 [batch+1]) live in host memory and may be reused by the
+ * caller as soon as the call returns. T == 0 returns HGX_OK without device work. */
+hgx_status hgx_attn_forward(hgx_attn_handle* h, void* stream, void* q, void* k, const void* v,
+                            void* out, const int32_t* pos_thw, const void* q_norm_w,
+                            const void* k_norm_w, int32_t batch, const int32_t* cu_seqlens_host,
+                            const hgx_segment* segs_host, const int32_t* cu_segs_host);
+
+/* The prologue alone on total_tokens tokens (q and k overwritten with q' and k'). */
+hgx_status hgx_attn_prologue(hgx_attn_handle* h, void* stream, void* q, void* k,
+                             const int32_t* pos_thw, const void* q_norm_w, const void* k_norm_w,
+                             int32_t total_tokens);
+
+/* The attention alone, on q and k that already hold q' and k' (nothing is overwritten). */
+hgx_status hgx_attn_attention(hgx_attn_handle* h, void* stream, const void* q, const void* k,
+                              const void* v, void* out, int32_t batch,
+                              const int32_t* cu_seqlens_host, const hgx_segment* segs_host,
+                              const int32_t* cu_segs_host);
+
+/* Host only (no GPU needed). Exclusive key limit lim(i) of every packed row, local to its
+ * batch element: row i sees keys [0, lim(i)). lim_out has room for cap entries; T entries
+ * are written. Errors: INVALID_ARG (descriptor, or cap < T). */
+hgx_status hgx_attn_row_limits(int32_t batch, const int32_t* cu_seqlens_host,
+                               const hgx_segment* segs_host, const int32_t* cu_segs_host,
+                               int32_t* lim_out, size_t cap);
+
+/* Host only. Tile classes at the attention kernel's real tile size: *bm_tokens query
+ * tokens (shared by all 4 query heads of a KV head) x *bn_keys keys. For each batch
+ * element in order, ceil(L/bm) x ceil(L/bn) bytes, row-major over (query block, key
+ * block), each an hgx_tile_class. Keys past the element's end count as masked, so a
+ * ragged last key block is never FULL. *n_written receives the number of bytes; if
+ * classes_out is NULL only the sizes are returned. */
+hgx_status hgx_attn_classify(int32_t batch, const int32_t* cu_seqlens_host,
+                             const hgx_segment* segs_host, const int32_t* cu_segs_host,
+                             int32_t* bm_tokens, int32_t* bn_keys, uint8_t* classes_out,
+                             size_t cap, size_t* n_written);
+
+/* Synchronizes `stream`, then reads and clears the handle's device error word: returns
+ * HGX_ERR_TIMEOUT if a bounded wait ran out since the last check, HGX_ERR_CUDA if the
+ * stream reports an error, HGX_OK otherwise. */
+hgx_status hgx_attn_sync_status(hgx_attn_handle* h, void* stream);
+
+/* Debug flags for hgx_attn_set_debug. */
+#define HGX_DEBUG_CHECKED 1u    /* every device call ends with hgx_attn_sync_status */
+#define HGX_DEBUG_STALL_TEST 2u /* attention: one softmax warpgroup first waits on a barrier
+                                   that nothing arrives at, so its bounded wait runs out */
+
+/* Sets debug flags and the bound of every device wait in nanoseconds (0 keeps the
+ * default of 2 s). The HGX_DEBUG environment variable (an integer) sets the initial
+ * flags of new handles. */
+hgx_status hgx_attn_set_debug(hgx_attn_handle* h, uint32_t flags, uint64_t wait_limit_ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HGX_ATTN_H */

@@ -1,0 +1,254 @@
+"""GPU parity of the sm_100a path against the fp64 oracle, through the C ABI.
+
+Tolerances (bf16 inputs, fp32 accumulation, unit-variance data): attention output
+max |err| <= 2e-2 and mean |err| <= 1e-3 against the fp64 oracle; the prologue's bf16
+q'/k' within bf16 rounding of the fp64 values (relative 2^-8 plus 1e-5 absolute for the
+fp32 arithmetic before rounding).
+
+Small configurations are compared element by element on every output; the full-size
+workloads (2048^2 text-to-image and edit, Hunyuan GCA) run in exactly the launch
+configuration the benchmark times and are compared on sampled rows that the oracle
+computes one by one (segment boundaries, tile edges, first and last rows, random rows).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+ATOL_MAX = 2e-2
+ATOL_MEAN = 1e-3
+
+
+@pytest.fixture(scope="module")
+def hgx():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    from unified_text_pixel_b200 import build
+
+    build.build()
+    import unified_text_pixel_b200 as H
+
+    a = H.Attention()
+    yield H, a
+    a.close()
+
+
+def _desc(w):
+    segs, cu_segs = W.flat_segments(w)
+    return W.cu_seqlens(w), segs, cu_segs
+
+
+def _device_inputs(w):
+    t = W.tensors(w)
+    d = {n: x.cuda() for n, x in t.items()}
+    d["pos"] = torch.from_numpy(W.positions(w)).cuda()
+    return t, d
+
+
+def _run(hgx, w, d=None):
+    H, a = hgx
+    if d is None:
+        _, d = _device_inputs(w)
+    out = torch.empty_like(d["q"])
+    a.forward(d["q"], d["k"], d["v"], out, d["pos"], d["wq"], d["wk"], *_desc(w))
+    assert a.sync_status() == H.HGX_OK
+    return out, d
+
+
+def _compare(got, ref, what):
+    err = np.abs(got.astype(np.float64) - ref)
+    assert np.isfinite(got).all(), what
+    assert err.max() <= ATOL_MAX, (what, float(err.max()))
+    assert err.mean() <= ATOL_MEAN, (what, float(err.mean()))
+    return float(err.max()), float(err.mean())
+
+
+def _oracle_full(w, t):
+    segs, cu_segs = W.flat_segments(w)
+    return O.forward(t["q"], t["k"], t["v"], W.positions(w), t["wq"], t["wk"], W.cu_seqlens(w), segs, cu_segs)
+
+
+# ------------------------------------------------------------------------------ prologue
+@pytest.mark.parametrize("case", ["c0", "c1", "ragged7", "one"])
+def test_prologue_matches_oracle(hgx, case):
+    H, a = hgx
+    w = {"c0": W.config(0), "c1": W.config(1), "ragged7": W.custom("r7", [[(3, 0), (4, 1)]], seed=11),
+         "one": W.custom("one", [[(1, 0)]], seed=12)}[case]
+    t, d = _device_inputs(w)
+    T = w.total_tokens
+    # canaries: one token row of padding on each side of q and k
+    qpad = torch.full((T + 2, 32, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+    kpad = torch.full((T + 2, 8, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+    qpad[1:-1] = d["q"]
+    kpad[1:-1] = d["k"]
+    a.prologue(qpad[1:-1], kpad[1:-1], d["pos"], d["wq"], d["wk"])
+    assert a.sync_status() == H.HGX_OK
+    qr, kr = O.prologue(t["q"], t["k"], W.positions(w), t["wq"], t["wk"])
+    for got, ref in ((qpad[1:-1], qr), (kpad[1:-1], kr)):
+        g = got.float().cpu().numpy().astype(np.float64)
+        np.testing.assert_allclose(g, ref, rtol=2.0 ** -8, atol=1e-5)
+    for pad in (qpad[0], qpad[-1], kpad[0], kpad[-1]):
+        assert bool((pad == 7.0).all())
+
+
+# ------------------------------------------------------------------------------ attention
+@pytest.mark.parametrize("cfg", [0, 1])
+def test_forward_small_configs_elementwise(hgx, cfg):
+    w = W.config(cfg)
+    t, _ = _device_inputs(w)
+    out, _ = _run(hgx, w)
+    ref, _, _ = _oracle_full(w, t)
+    _compare(out.float().cpu().numpy(), ref, w.name)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_forward_random_layouts_elementwise(hgx, seed):
+    """Ragged lengths, all three kinds, several batch elements, empty elements."""
+    w = W.random_workload(100 + seed, max_batch=4, max_len=520, allow_empty=True)
+    if w.total_tokens == 0:
+        pytest.skip("empty draw")
+    t, _ = _device_inputs(w)
+    out, _ = _run(hgx, w)
+    ref, _, _ = _oracle_full(w, t)
+    _compare(out.float().cpu().numpy(), ref, w.name)
+
+
+def test_attention_alone_on_kernel_rotated_inputs(hgx):
+    """The attention kernel against the oracle's masked softmax applied to the very bf16
+    q'/k' the prologue kernel wrote (isolates attention error from prologue rounding)."""
+    H, a = hgx
+    w = W.config(1)
+    t, d = _device_inputs(w)
+    a.prologue(d["q"], d["k"], d["pos"], d["wq"], d["wk"])
+    out = torch.empty_like(d["q"])
+    a.attention(d["q"], d["k"], d["v"], out, *_desc(w))
+    assert a.sync_status() == H.HGX_OK
+    qp = d["q"].float().cpu().numpy().astype(np.float64)
+    kp = d["k"].float().cpu().numpy().astype(np.float64)
+    vv = t["v"].float().numpy().astype(np.float64)
+    cu, segs, cu_segs = _desc(w)
+    got = out.float().cpu().numpy()
+    for b in range(len(cu) - 1):
+        t0, t1 = int(cu[b]), int(cu[b + 1])
+        bsegs = [tuple(int(x) for x in segs[n]) for n in range(cu_segs[b], cu_segs[b + 1])]
+        ref = O.masked_gqa_attention(qp[t0:t1], kp[t0:t1], vv[t0:t1], O.dense_mask(bsegs, t1 - t0))
+        err = np.abs(got[t0:t1] - ref)
+        assert err.max() <= 1e-2 and err.mean() <= 5e-4, (float(err.max()), float(err.mean()))
+
+
+def test_single_token_returns_its_value(hgx):
+    """One causal token sees only itself: out[0, h] == v[0, h // 4] (rounded to bf16)."""
+    w = W.custom("one", [[(1, W.CAUSAL)]], seed=5)
+    t, _ = _device_inputs(w)
+    out, _ = _run(hgx, w)
+    v = t["v"].float()
+    for h in range(32):
+        torch.testing.assert_close(out[0, h].float().cpu(), v[0, h // 4], rtol=2 ** -8, atol=1e-6)
+
+
+def _sample_rows(w, n_random=24, seed=0):
+    rows = set()
+    cu = W.cu_seqlens(w)
+    for b, batch in enumerate(w.batches):
+        base, L = int(cu[b]), w.lengths[b]
+        for s in batch:
+            for r in (s.start - 1, s.start, s.start + 1, s.start + s.length - 1):
+                if 0 <= r < L:
+                    rows.add(base + r)
+        for edge in range(0, L, 2048):
+            for r in (edge - 1, edge, edge + 31, edge + 32, edge + 63, edge + 64, edge + 127, edge + 128):
+                if 0 <= r < L:
+                    rows.add(base + r)
+        rows.update({base, base + L - 1})
+    rng = np.random.default_rng(seed)
+    rows.update(int(x) for x in rng.integers(0, w.total_tokens, size=n_random))
+    return sorted(rows)
+
+
+@pytest.mark.parametrize("cfg", [2, 3, 4])
+def test_forward_full_size_sampled_rows(hgx, cfg):
+    w = W.config(cfg)
+    t, _ = _device_inputs(w)
+    out, _ = _run(hgx, w)
+    rows = _sample_rows(w, seed=cfg)
+    segs, cu_segs = W.flat_segments(w)
+    ref = O.attention_rows(t["q"], t["k"], t["v"], W.positions(w), t["wq"], t["wk"], W.cu_seqlens(w), segs,
+                           cu_segs, rows)
+    got = out[rows].float().cpu().numpy()
+    _compare(got, ref, w.name)
+    assert torch.isfinite(out.float()).all()
+
+
+def test_forward_is_deterministic(hgx):
+    w = W.config(1)
+    _, d0 = _device_inputs(w)
+    _, d1 = _device_inputs(w)
+    o0, _ = _run(hgx, w, d0)
+    o1, _ = _run(hgx, w, d1)
+    assert torch.equal(o0, o1)
+
+
+def test_output_canaries_untouched(hgx):
+    H, a = hgx
+    w = W.random_workload(7, max_batch=3, max_len=300)
+    _, d = _device_inputs(w)
+    T = w.total_tokens
+    pad = torch.full((T + 2, 32, 128), -3.0, dtype=torch.bfloat16, device="cuda")
+    a.forward(d["q"], d["k"], d["v"], pad[1:-1], d["pos"], d["wq"], d["wk"], *_desc(w))
+    assert a.sync_status() == H.HGX_OK
+    assert bool((pad[0] == -3.0).all()) and bool((pad[-1] == -3.0).all())
+    assert torch.isfinite(pad[1:-1].float()).all()
+
+
+def test_maximum_token_count_sampled(hgx):
+    """The largest packed size the ABI accepts (2^19 - 1 tokens, 128 batch elements):
+    exercises the highest byte offsets; sampled rows of the last elements."""
+    H, a = hgx
+    n_el, per = 128, 4096
+    total = (1 << 19) - 1
+    lens = [per] * (n_el - 1) + [total - per * (n_el - 1)]
+    batches = []
+    for i, L in enumerate(lens):
+        kinds = [(L // 4, W.CAUSAL), (L // 2, [W.FULL_SEQUENCE, W.FULL_IN_SEGMENT][i % 2]),
+                 (L - L // 4 - L // 2, W.CAUSAL)]
+        batches.append(kinds)
+    w = W.custom("max_tokens", batches, seed=21)
+    assert w.total_tokens == total
+    t, _ = _device_inputs(w)
+    out, _ = _run(hgx, w)
+    cu = W.cu_seqlens(w)
+    rows = [int(cu[-2]) + r for r in (0, 1, 1023, 1024, 3000, lens[-1] - 1)] + [int(cu[60]) + 5, total - 1]
+    segs, cu_segs = W.flat_segments(w)
+    ref = O.attention_rows(t["q"], t["k"], t["v"], W.positions(w), t["wq"], t["wk"], cu, segs, cu_segs, rows)
+    _compare(out[rows].float().cpu().numpy(), ref, "max_tokens")
+
+
+def test_empty_batch_is_a_no_op(hgx):
+    H, a = hgx
+    z = torch.zeros(1, dtype=torch.bfloat16, device="cuda")
+    a.forward(z, z, z, z, z, z, z, [0, 0], np.zeros((0, 3)), [0, 0])
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(hgx):
+    """A softmax warpgroup waits on a barrier that nothing arrives at; its bounded wait
+    runs out, the kernel drains and exits, the host sees HGX_ERR_TIMEOUT, and the next
+    normal call on the same context is correct."""
+    H, a = hgx
+    w = W.config(0)
+    t, d = _device_inputs(w)
+    out = torch.empty_like(d["q"])
+    q0, k0 = d["q"].clone(), d["k"].clone()
+    a.set_debug(H.HGX_DEBUG_STALL_TEST | H.HGX_DEBUG_CHECKED, 20_000_000)
+    with pytest.raises(H.HgxError) as e:
+        a.forward(d["q"], d["k"], d["v"], out, d["pos"], d["wq"], d["wk"], *_desc(w))
+    assert e.value.status == H.HGX_ERR_TIMEOUT
+    a.set_debug(0, 0)
+    d["q"].copy_(q0)
+    d["k"].copy_(k0)
+    out, _ = _run(hgx, w, d)
+    ref, _, _ = _oracle_full(w, t)
+    _compare(out.float().cpu().numpy(), ref, "after-timeout")

@@ -1,0 +1,205 @@
+"""Host planner and C ABI, on the CPU (no GPU, no kernel launches).
+
+* per-row key limits and tile classes from the library's planner against the oracle's
+  dense mask (built from the segment rules, never through limits): bit-exact;
+* descriptor validation: every malformed request returns its documented status before
+  any device work;
+* the shared library loads and exports every function that include/hgx_attn.h declares.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle as O
+import workloads as W
+from unified_text_pixel_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built_library():
+    from unified_text_pixel_b200 import build
+
+    build.build()
+
+
+def _desc(w):
+    segs, cu_segs = W.flat_segments(w)
+    return W.cu_seqlens(w), segs, cu_segs
+
+
+def _check_against_mask(w):
+    cu, segs, cu_segs = _desc(w)
+    lim = B.row_limits(cu, segs, cu_segs)
+    bm, bn, classes = B.classify(cu, segs, cu_segs)
+    at = 0
+    for b in range(len(cu) - 1):
+        t0, t1 = int(cu[b]), int(cu[b + 1])
+        L = t1 - t0
+        bsegs = [tuple(int(x) for x in segs[n]) for n in range(cu_segs[b], cu_segs[b + 1])]
+        mask = O.dense_mask(bsegs, L)
+        # every row's visible set is exactly the prefix [0, lim)
+        expect = np.zeros_like(mask)
+        for i in range(L):
+            expect[i, : lim[t0 + i]] = True
+        np.testing.assert_array_equal(mask, expect)
+        ref = O.tile_classes(mask, bm, bn)
+        got = classes[at : at + ref.size].reshape(ref.shape)
+        at += ref.size
+        np.testing.assert_array_equal(got, ref)
+    assert at == classes.size
+
+
+@pytest.mark.parametrize("cfg", range(5))
+def test_limits_and_tile_classes_match_dense_mask(cfg):
+    _check_against_mask(W.config(cfg))
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_limits_and_tile_classes_random_layouts(seed):
+    _check_against_mask(W.random_workload(seed, allow_empty=(seed % 5 == 0)))
+
+
+def test_tile_size_is_the_kernels():
+    bm, bn, _ = B.classify(*_desc(W.config(0)))
+    assert (bm, bn) == (64, 128)
+
+
+def test_visible_pairs_match_closed_forms():
+    from conftest import read_golden
+
+    rows = {ln.split()[0]: int(ln.split()[1]) for ln in read_golden("unmasked_pairs.txt")}
+    for w in W.CONFIGS:
+        assert int(B.row_limits(*_desc(w)).astype(np.int64).sum()) == rows[w.name]
+
+
+# ----------------------------------------------------------------------------- validation
+def _status_row_limits(cu, segs, cu_segs):
+    cu, sg, cs = B._descriptor(cu, segs, cu_segs)
+    out = np.zeros(max(1, int(cu[-1]) if cu.size else 1), dtype=np.int32)
+    return B.lib().hgx_attn_row_limits(len(cu) - 1, B._ptr(cu), B._ptr(sg), B._ptr(cs), B._ptr(out), out.size)
+
+
+BAD = {
+    "bad_kind": ([0, 5], [[0, 5, 3]], [0, 1]),
+    "negative_kind": ([0, 5], [[0, 5, -1]], [0, 1]),
+    "gap": ([0, 5], [[0, 2, 0], [3, 2, 1]], [0, 2]),
+    "overlap": ([0, 5], [[0, 3, 0], [2, 3, 1]], [0, 2]),
+    "zero_len": ([0, 5], [[0, 0, 0], [0, 5, 1]], [0, 2]),
+    "short": ([0, 5], [[0, 4, 0]], [0, 1]),
+    "long": ([0, 5], [[0, 6, 0]], [0, 1]),
+    "cu_decreasing": ([0, 5, 3], [[0, 5, 0]], [0, 1, 1]),
+    "cu_nonzero_start": ([1, 5], [[0, 4, 0]], [0, 1]),
+    "too_many_tokens": ([0, 1 << 19], [[0, 1 << 19, 1]], [0, 1]),
+    "segments_for_empty": ([0, 0], [[0, 1, 0]], [0, 1]),
+}
+
+
+@pytest.mark.parametrize("name", sorted(BAD))
+def test_malformed_descriptors_rejected(name):
+    assert _status_row_limits(*BAD[name]) == B.HGX_ERR_INVALID_ARG
+
+
+def test_empty_batch_element_is_valid():
+    lim = B.row_limits([0, 0, 3], [[0, 3, 1]], [0, 0, 1])
+    assert list(lim) == [3, 3, 3]
+
+
+def test_create_rejects_bad_configs():
+    L = B.lib()
+    base = B.Attention.default_config()
+
+    def status(**kw):
+        cfg = B.AttnConfig()
+        ctypes.pointer(cfg)[0] = base
+        for k, v in kw.items():
+            if k == "mrope_section":
+                cfg.mrope_section[:] = v
+            else:
+                setattr(cfg, k, v)
+        h = ctypes.c_void_p()
+        st = L.hgx_attn_create(ctypes.byref(cfg), ctypes.byref(h))
+        if h.value:
+            L.hgx_attn_destroy(h)
+        return st
+
+    assert status() == B.HGX_OK
+    assert status(num_q_heads=16) == B.HGX_ERR_UNSUPPORTED
+    assert status(head_dim=64) == B.HGX_ERR_UNSUPPORTED
+    assert status(num_kv_heads=0) == B.HGX_ERR_INVALID_ARG
+    assert status(rope_theta=-1.0) == B.HGX_ERR_INVALID_ARG
+    assert status(rms_eps=-1.0) == B.HGX_ERR_INVALID_ARG
+    assert status(mrope_section=[24, 20, 21]) == B.HGX_ERR_INVALID_ARG
+    assert status(mrope_section=[4, 30, 30]) == B.HGX_ERR_UNSUPPORTED
+    assert L.hgx_attn_create(None, ctypes.byref(ctypes.c_void_p())) == B.HGX_ERR_INVALID_ARG
+
+
+def _fake(addr):
+    # a non-null host integer posing as a device pointer: these calls must fail before
+    # anything dereferences it
+    class P:
+        def data_ptr(self):
+            return addr
+
+    return P()
+
+
+def test_forward_rejects_before_device_work():
+    a = B.Attention()
+    cu, segs, cu_segs = [0, 8], [[0, 8, 0]], [0, 1]
+    good = [_fake(0x10000 * (i + 1)) for i in range(7)]
+    # malformed descriptor
+    with pytest.raises(B.HgxError) as e:
+        a.forward(*good, [0, 8], [[0, 7, 0]], [0, 1], stream=0)
+    assert e.value.status == B.HGX_ERR_INVALID_ARG
+    # null pointer
+    for i in range(7):
+        args = list(good)
+        args[i] = None
+        with pytest.raises(B.HgxError) as e:
+            a.forward(*args, cu, segs, cu_segs, stream=0)
+        assert e.value.status == B.HGX_ERR_INVALID_ARG
+    # misaligned pointer
+    args = list(good)
+    args[2] = _fake(0x30008)
+    with pytest.raises(B.HgxError) as e:
+        a.forward(*args, cu, segs, cu_segs, stream=0)
+    assert e.value.status == B.HGX_ERR_INVALID_ARG and "aligned" in str(e.value)
+    # out overlapping q
+    args = list(good)
+    args[3] = _fake(0x10000 + 4096)
+    with pytest.raises(B.HgxError) as e:
+        a.forward(*args, cu, segs, cu_segs, stream=0)
+    assert e.value.status == B.HGX_ERR_INVALID_ARG and "overlap" in str(e.value)
+    # an empty batch returns OK without touching the device (works without a GPU)
+    a.forward(*[None] * 7, [0, 0], np.zeros((0, 3)), [0, 0], stream=0)
+    a.close()
+
+
+def test_set_debug_rejects_unknown_flags():
+    a = B.Attention()
+    with pytest.raises(B.HgxError):
+        a.set_debug(0x80)
+    a.set_debug(B.HGX_DEBUG_CHECKED, 10_000_000)
+    a.close()
+
+
+def test_library_exports_every_declared_symbol():
+    with open(os.path.join(ROOT, "include", "hgx_attn.h")) as f:
+        text = f.read()
+    declared = sorted(set(re.findall(r"\b(hgx_attn_\w+)\s*\(", text)))
+    assert len(declared) >= 11
+    L = ctypes.CDLL(B.library_path)
+    for name in declared:
+        assert hasattr(L, name), name
+
+
+def test_binding_raises_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(B, "library_path", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(B, "_lib", None)
+    with pytest.raises(B.HgxError):
+        B.lib()

@@ -1,0 +1,206 @@
+"""ctypes binding of libhgx_attn.so: argument marshalling only.
+
+Tensors are passed as raw device pointers (torch is used for device memory and streams);
+segment descriptors are passed as host int32 arrays. Every step of the path runs in the
+library's kernels.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence, Tuple
+
+import numpy as np
+
+HGX_OK, HGX_ERR_INVALID_ARG, HGX_ERR_UNSUPPORTED, HGX_ERR_OOM, HGX_ERR_CUDA, HGX_ERR_TIMEOUT = range(6)
+HGX_SEG_CAUSAL, HGX_SEG_FULL_SEQUENCE, HGX_SEG_FULL_IN_SEGMENT = 0, 1, 2
+HGX_TILE_SKIP, HGX_TILE_PARTIAL, HGX_TILE_FULL = 0, 1, 2
+HGX_DEBUG_CHECKED, HGX_DEBUG_STALL_TEST = 1, 2
+
+_STATUS = {0: "HGX_OK", 1: "HGX_ERR_INVALID_ARG", 2: "HGX_ERR_UNSUPPORTED", 3: "HGX_ERR_OOM",
+           4: "HGX_ERR_CUDA", 5: "HGX_ERR_TIMEOUT"}
+
+library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhgx_attn.so")
+
+
+class HgxError(RuntimeError):
+    def __init__(self, status: int, message: str = ""):
+        self.status = status
+        super().__init__(f"{_STATUS.get(status, status)}: {message}")
+
+
+class AttnConfig(ctypes.Structure):
+    _fields_ = [
+        ("num_q_heads", ctypes.c_int32),
+        ("num_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("rope_theta", ctypes.c_double),
+        ("mrope_section", ctypes.c_int32 * 3),
+        ("rms_eps", ctypes.c_float),
+        ("softmax_scale", ctypes.c_float),
+    ]
+
+
+_lib = None
+
+_SIGS = {
+    "hgx_attn_default_config": (None, [ctypes.c_void_p]),
+    "hgx_attn_create": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_void_p)]),
+    "hgx_attn_destroy": (None, [ctypes.c_void_p]),
+    "hgx_attn_last_error": (ctypes.c_char_p, [ctypes.c_void_p]),
+    "hgx_attn_forward": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_int32] + [ctypes.c_void_p] * 3),
+    "hgx_attn_prologue": (ctypes.c_int, [ctypes.c_void_p] * 7 + [ctypes.c_int32]),
+    "hgx_attn_attention": (ctypes.c_int, [ctypes.c_void_p] * 6 + [ctypes.c_int32] + [ctypes.c_void_p] * 3),
+    "hgx_attn_row_limits": (ctypes.c_int, [ctypes.c_int32] + [ctypes.c_void_p] * 4 + [ctypes.c_size_t]),
+    "hgx_attn_classify": (ctypes.c_int, [ctypes.c_int32] + [ctypes.c_void_p] * 6 + [ctypes.c_size_t, ctypes.c_void_p]),
+    "hgx_attn_sync_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
+    "hgx_attn_set_debug": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_uint32, ctypes.c_uint64]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libhgx_attn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(library_path):
+            raise HgxError(HGX_ERR_UNSUPPORTED, f"{library_path} is missing: run "
+                           "`python -m unified_text_pixel_b200.build` (there is no fallback)")
+        L = ctypes.CDLL(library_path)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _i32(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int32))
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p) if a.size else None
+
+
+def _descriptor(cu_seqlens, segs, cu_segs):
+    cu = _i32(cu_seqlens).reshape(-1)
+    sg = _i32(segs).reshape(-1, 3)
+    cs = _i32(cu_segs).reshape(-1)
+    return cu, sg, cs
+
+
+def row_limits(cu_seqlens, segs, cu_segs) -> np.ndarray:
+    """Exclusive key limit of every packed row (host-side planner of the library)."""
+    cu, sg, cs = _descriptor(cu_seqlens, segs, cu_segs)
+    T = int(cu[-1]) if cu.size else 0
+    out = np.zeros(T, dtype=np.int32)
+    st = lib().hgx_attn_row_limits(len(cu) - 1, _ptr(cu), _ptr(sg), _ptr(cs), _ptr(out), T)
+    if st != HGX_OK:
+        raise HgxError(st, "hgx_attn_row_limits")
+    return out
+
+
+def classify(cu_seqlens, segs, cu_segs) -> Tuple[int, int, np.ndarray]:
+    """(bm_tokens, bn_keys, classes uint8) at the attention kernel's tile size."""
+    cu, sg, cs = _descriptor(cu_seqlens, segs, cu_segs)
+    bm, bn, n = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_size_t()
+    L = lib()
+    st = L.hgx_attn_classify(len(cu) - 1, _ptr(cu), _ptr(sg), _ptr(cs), ctypes.byref(bm),
+                             ctypes.byref(bn), None, 0, ctypes.byref(n))
+    if st != HGX_OK:
+        raise HgxError(st, "hgx_attn_classify")
+    out = np.zeros(n.value, dtype=np.uint8)
+    st = L.hgx_attn_classify(len(cu) - 1, _ptr(cu), _ptr(sg), _ptr(cs), ctypes.byref(bm),
+                             ctypes.byref(bn), _ptr(out), out.size, ctypes.byref(n))
+    if st != HGX_OK:
+        raise HgxError(st, "hgx_attn_classify")
+    return bm.value, bn.value, out
+
+
+def _dev_ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream):
+    """torch.cuda.Stream, a raw cudaStream_t integer, or None for torch's current stream."""
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    if stream is None:
+        import torch
+
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+class Attention:
+    """Owns one hgx_attn_handle. Methods take torch CUDA tensors (bf16 / int32)."""
+
+    def __init__(self, config: Optional[AttnConfig] = None):
+        L = lib()
+        cfg = AttnConfig()
+        L.hgx_attn_default_config(ctypes.byref(cfg))
+        if config is not None:
+            cfg = config
+        self.config = cfg
+        h = ctypes.c_void_p()
+        st = L.hgx_attn_create(ctypes.byref(cfg), ctypes.byref(h))
+        if st != HGX_OK:
+            raise HgxError(st, "hgx_attn_create")
+        self._h = h
+
+    @staticmethod
+    def default_config() -> AttnConfig:
+        cfg = AttnConfig()
+        lib().hgx_attn_default_config(ctypes.byref(cfg))
+        return cfg
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib().hgx_attn_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def _check(self, st: int, what: str):
+        if st != HGX_OK:
+            msg = lib().hgx_attn_last_error(self._h) or b""
+            raise HgxError(st, f"{what}: {msg.decode(errors='replace')}")
+
+    def forward(self, q, k, v, out, pos, wq, wk, cu_seqlens, segs, cu_segs, stream=None):
+        """hgx_attn_forward: q, k overwritten with q', k'; out written."""
+        cu, sg, cs = _descriptor(cu_seqlens, segs, cu_segs)
+        st = lib().hgx_attn_forward(self._h, _stream_ptr(stream), _dev_ptr(q), _dev_ptr(k), _dev_ptr(v),
+                                    _dev_ptr(out), _dev_ptr(pos), _dev_ptr(wq), _dev_ptr(wk), len(cu) - 1,
+                                    _ptr(cu), _ptr(sg), _ptr(cs))
+        self._check(st, "hgx_attn_forward")
+
+    def prologue(self, q, k, pos, wq, wk, total_tokens=None, stream=None):
+        T = q.shape[0] if total_tokens is None else total_tokens
+        st = lib().hgx_attn_prologue(self._h, _stream_ptr(stream), _dev_ptr(q), _dev_ptr(k), _dev_ptr(pos),
+                                     _dev_ptr(wq), _dev_ptr(wk), int(T))
+        self._check(st, "hgx_attn_prologue")
+
+    def attention(self, q, k, v, out, cu_seqlens, segs, cu_segs, stream=None):
+        cu, sg, cs = _descriptor(cu_seqlens, segs, cu_segs)
+        st = lib().hgx_attn_attention(self._h, _stream_ptr(stream), _dev_ptr(q), _dev_ptr(k), _dev_ptr(v),
+                                      _dev_ptr(out), len(cu) - 1, _ptr(cu), _ptr(sg), _ptr(cs))
+        self._check(st, "hgx_attn_attention")
+
+    def sync_status(self, stream=None) -> int:
+        """Synchronizes the stream; returns the status code (HGX_ERR_TIMEOUT after a wait ran out)."""
+        return lib().hgx_attn_sync_status(self._h, _stream_ptr(stream))
+
+    def set_debug(self, flags: int, wait_limit_ns: int = 0):
+        self._check(lib().hgx_attn_set_debug(self._h, flags, wait_limit_ns), "hgx_attn_set_debug")
+
+    def last_error(self) -> str:
+        return (lib().hgx_attn_last_error(self._h) or b"").decode(errors="replace")
+
+    # raw access for ABI tests
+    @property
+    def handle(self):
+        return self._h

@@ -1,0 +1,459 @@
+// C ABI of the hybrid-masked attention (declared in include/hgx_attn.h).
+//
+// Every argument is checked on the host before any device work, as the HiDream-O1 port
+// does for contract errors ("hidream-o1-p100a" model card, "Serving (HTTP)": rejected
+// without touching the card). The handle caches the plan (row limits, work list) of the
+// last segment descriptor and re-uploads it only when the descriptor changes.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/hgx_attn.h"
+#include "kernels.h"
+#include "planner.h"
+
+struct hgx_attn_handle {
+  hgx_attn_config cfg{};
+  float scale = 0.f;
+  hgx::RopeTables rope{};
+  std::string last_error;
+  uint32_t flags = 0;
+  uint64_t wait_limit_ns = 2000000000ull;
+
+  // cached descriptor and its plan
+  int32_t key_batch = -1;
+  std::vector<int32_t> key_cu, key_cu_segs;
+  std::vector<hgx_segment> key_segs;
+  hgx::Plan plan;
+  int plan_device = -1;
+
+  // device scratch owned by the handle
+  int device = -1;
+  int num_sms = 0;
+  int32_t* d_lim = nullptr;
+  size_t lim_cap = 0;
+  hgx::WorkItem* d_items = nullptr;
+  size_t items_cap = 0;
+  uint32_t* d_err = nullptr;
+  // pinned staging for the plan upload, reused once the previous upload has completed
+  uint8_t* h_stage = nullptr;
+  size_t stage_cap = 0;
+  cudaEvent_t stage_done = nullptr;
+};
+
+namespace {
+
+using PFN_encodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                     const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                     const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                     CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+hgx_status fail(hgx_attn_handle* h, hgx_status st, const std::string& msg) {
+  if (h) h->last_error = msg;
+  return st;
+}
+
+hgx_status cuda_fail(hgx_attn_handle* h, cudaError_t e, const char* what) {
+  return fail(h, HGX_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+PFN_encodeTiled encode_fn() {
+  static PFN_encodeTiled fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_encodeTiled>(ptr);
+  }
+  return fn;
+}
+
+// 3-D bf16 tensor map over [T, heads, 128] with a box of (64 features, box_heads,
+// box_tokens) and 128-byte swizzle; boxes past T read zeros.
+bool make_map(CUtensorMap* map, const void* ptr, int heads, int T, int box_heads,
+              int box_tokens) {
+  PFN_encodeTiled enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(heads), static_cast<cuuint64_t>(T)};
+  cuuint64_t strides[2] = {256, static_cast<cuuint64_t>(heads) * 256};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_heads),
+                       static_cast<cuuint32_t>(box_tokens)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+hgx_status ensure_device(hgx_attn_handle* h) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(h, e, "cudaGetDevice");
+  if (h->device == dev) return HGX_OK;
+  if (h->device >= 0) return fail(h, HGX_ERR_INVALID_ARG, "handle is bound to another device");
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0)
+    return fail(h, HGX_ERR_UNSUPPORTED, "this library is built for sm_100a (B200) only");
+  e = cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(h, e, "cudaDeviceGetAttribute");
+  e = cudaMalloc(&h->d_err, sizeof(uint32_t));
+  if (e != cudaSuccess) return fail(h, HGX_ERR_OOM, "cudaMalloc of the error word failed");
+  e = cudaMemset(h->d_err, 0, sizeof(uint32_t));
+  if (e != cudaSuccess) return cuda_fail(h, e, "cudaMemset");
+  e = cudaEventCreateWithFlags(&h->stage_done, cudaEventDisableTiming);
+  if (e != cudaSuccess) return cuda_fail(h, e, "cudaEventCreate");
+  h->device = dev;
+  return HGX_OK;
+}
+
+bool same_descriptor(const hgx_attn_handle* h, int32_t batch, const int32_t* cu,
+                     const hgx_segment* segs, const int32_t* cu_segs) {
+  if (h->key_batch != batch) return false;
+  if (std::memcmp(h->key_cu.data(), cu, sizeof(int32_t) * (batch + 1)) != 0) return false;
+  if (std::memcmp(h->key_cu_segs.data(), cu_segs, sizeof(int32_t) * (batch + 1)) != 0)
+    return false;
+  const size_t ns = static_cast<size_t>(cu_segs[batch]);
+  if (h->key_segs.size() != ns) return false;
+  return ns == 0 || std::memcmp(h->key_segs.data(), segs, sizeof(hgx_segment) * ns) == 0;
+}
+
+// Builds (or reuses) the plan of this descriptor and makes sure it is on the device,
+// uploaded in stream order.
+hgx_status prepare_plan(hgx_attn_handle* h, cudaStream_t stream, int32_t batch,
+                        const int32_t* cu, const hgx_segment* segs, const int32_t* cu_segs) {
+  const bool same = same_descriptor(h, batch, cu, segs, cu_segs);
+  if (!same) {
+    hgx::Plan plan;
+    std::string err;
+    hgx_status st = hgx::build_plan(batch, cu, segs, cu_segs, h->cfg.num_kv_heads, &plan, &err);
+    if (st != HGX_OK) return fail(h, st, err);
+    h->plan = std::move(plan);
+    h->key_batch = batch;
+    h->key_cu.assign(cu, cu + batch + 1);
+    h->key_cu_segs.assign(cu_segs, cu_segs + batch + 1);
+    h->key_segs.assign(segs, segs + cu_segs[batch]);
+    h->plan_device = -1;
+  }
+  if (h->plan_device == h->device) return HGX_OK;
+  const size_t T = static_cast<size_t>(h->plan.total_tokens);
+  const size_t n_items = h->plan.items.size();
+  cudaError_t e;
+  if (T > h->lim_cap) {
+    if (h->d_lim) cudaFree(h->d_lim);
+    h->d_lim = nullptr;
+    h->lim_cap = 0;
+    if (cudaMalloc(&h->d_lim, T * sizeof(int32_t)) != cudaSuccess)
+      return fail(h, HGX_ERR_OOM, "cudaMalloc of the row limits failed");
+    h->lim_cap = T;
+  }
+  if (n_items > h->items_cap) {
+    if (h->d_items) cudaFree(h->d_items);
+    h->d_items = nullptr;
+    h->items_cap = 0;
+    if (cudaMalloc(&h->d_items, n_items * sizeof(hgx::WorkItem)) != cudaSuccess)
+      return fail(h, HGX_ERR_OOM, "cudaMalloc of the work list failed");
+    h->items_cap = n_items;
+  }
+  const size_t lim_bytes = T * sizeof(int32_t);
+  const size_t item_off = (lim_bytes + 255) & ~size_t(255);
+  const size_t need = item_off + n_items * sizeof(hgx::WorkItem);
+  // the previous upload may still be reading the staging buffer
+  e = cudaEventSynchronize(h->stage_done);
+  if (e != cudaSuccess) return cuda_fail(h, e, "cudaEventSynchronize");
+  if (need > h->stage_cap) {
+    if (h->h_stage) cudaFreeHost(h->h_stage);
+    h->h_stage = nullptr;
+    h->stage_cap = 0;
+    if (cudaMallocHost(&h->h_stage, need) != cudaSuccess)
+      return fail(h, HGX_ERR_OOM, "cudaMallocHost of the plan staging buffer failed");
+    h->stage_cap = need;
+  }
+  std::memcpy(h->h_stage, h->plan.lim.data(), lim_bytes);
+  std::memcpy(h->h_stage + item_off, h->plan.items.data(), n_items * sizeof(hgx::WorkItem));
+  if (lim_bytes) {
+    e = cudaMemcpyAsync(h->d_lim, h->h_stage, lim_bytes, cudaMemcpyHostToDevice, stream);
+    if (e != cudaSuccess) return cuda_fail(h, e, "cudaMemcpyAsync (row limits)");
+  }
+  if (n_items) {
+    e = cudaMemcpyAsync(h->d_items, h->h_stage + item_off, n_items * sizeof(hgx::WorkItem),
+                        cudaMemcpyHostToDevice, stream);
+    if (e != cudaSuccess) return cuda_fail(h, e, "cudaMemcpyAsync (work list)");
+  }
+  e = cudaEventRecord(h->stage_done, stream);
+  if (e != cudaSuccess) return cuda_fail(h, e, "cudaEventRecord");
+  h->plan_device = h->device;
+  return HGX_OK;
+}
+
+hgx_status check_tensors(hgx_attn_handle* h, std::initializer_list<const void*> ptrs) {
+  for (const void* p : ptrs) {
+    if (!p) return fail(h, HGX_ERR_INVALID_ARG, "device pointer is NULL");
+    if (!aligned16(p)) return fail(h, HGX_ERR_INVALID_ARG, "device pointer is not 16-byte aligned");
+  }
+  return HGX_OK;
+}
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+hgx_status finish(hgx_attn_handle* h, cudaStream_t stream) {
+  if (h->flags & HGX_DEBUG_CHECKED) return hgx_attn_sync_status(h, stream);
+  return HGX_OK;
+}
+
+hgx_status run_attention(hgx_attn_handle* h, cudaStream_t stream, const void* q, const void* k,
+                         const void* v, void* out) {
+  const int32_t T = h->plan.total_tokens;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, 32, T, 4, hgx::kTileTokens) || !make_map(&mk, k, 8, T, 1, 128) ||
+      !make_map(&mv, v, 8, T, 1, 128))
+    return fail(h, HGX_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  hgx::AttnParams p{};
+  p.items = h->d_items;
+  p.n_items = static_cast<int32_t>(h->plan.items.size());
+  p.total_tokens = T;
+  p.lim = h->d_lim;
+  p.out = out;
+  p.scale_log2 = h->scale * 1.4426950408889634f;
+  p.flags = h->flags;
+  p.err = h->d_err;
+  p.wait_limit_ns = h->wait_limit_ns;
+  const int grid = p.n_items < h->num_sms ? p.n_items : h->num_sms;
+  cudaError_t e = hgx::launch_attention(stream, mq, mk, mv, p, grid);
+  if (e != cudaSuccess) return cuda_fail(h, e, "attention launch");
+  return HGX_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+void hgx_attn_default_config(hgx_attn_config* cfg) {
+  if (!cfg) return;
+  cfg->num_q_heads = 32;
+  cfg->num_kv_heads = 8;
+  cfg->head_dim = 128;
+  cfg->rope_theta = 5.0e6;
+  cfg->mrope_section[0] = 24;
+  cfg->mrope_section[1] = 20;
+  cfg->mrope_section[2] = 20;
+  cfg->rms_eps = 1e-6f;
+  cfg->softmax_scale = 0.f;
+}
+
+hgx_status hgx_attn_create(const hgx_attn_config* cfg, hgx_attn_handle** out) {
+  if (!out) return HGX_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!cfg) return HGX_ERR_INVALID_ARG;
+  if (!(cfg->rope_theta > 0.0) || !std::isfinite(cfg->rope_theta)) return HGX_ERR_INVALID_ARG;
+  if (!(cfg->rms_eps >= 0.f) || !std::isfinite(cfg->rms_eps)) return HGX_ERR_INVALID_ARG;
+  if (!(cfg->softmax_scale >= 0.f) || !std::isfinite(cfg->softmax_scale))
+    return HGX_ERR_INVALID_ARG;
+  for (int i = 0; i < 3; ++i)
+    if (cfg->mrope_section[i] < 0) return HGX_ERR_INVALID_ARG;
+  if (cfg->num_q_heads <= 0 || cfg->num_kv_heads <= 0 || cfg->head_dim <= 0)
+    return HGX_ERR_INVALID_ARG;
+  if (cfg->num_q_heads != 32 || cfg->num_kv_heads != 8 || cfg->head_dim != 128)
+    return HGX_ERR_UNSUPPORTED;
+  if (cfg->mrope_section[0] + cfg->mrope_section[1] + cfg->mrope_section[2] != cfg->head_dim / 2)
+    return HGX_ERR_INVALID_ARG;
+  {
+    // the interleaved assignment must give each axis exactly its section's count
+    double inv[64];
+    int32_t axis[64], count[3] = {0, 0, 0};
+    hgx::mrope_tables(cfg->rope_theta, cfg->head_dim, cfg->mrope_section, inv, axis);
+    for (int i = 0; i < 64; ++i) ++count[axis[i]];
+    for (int i = 0; i < 3; ++i)
+      if (count[i] != cfg->mrope_section[i]) return HGX_ERR_UNSUPPORTED;
+  }
+  hgx_attn_handle* h = new (std::nothrow) hgx_attn_handle();
+  if (!h) return HGX_ERR_OOM;
+  h->cfg = *cfg;
+  h->scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale
+                                      : static_cast<float>(1.0 / std::sqrt(double(cfg->head_dim)));
+  int32_t axis[64];
+  hgx::mrope_tables(cfg->rope_theta, cfg->head_dim, cfg->mrope_section, h->rope.inv_freq, axis);
+  for (int i = 0; i < 64; ++i) h->rope.axis[i] = static_cast<uint8_t>(axis[i]);
+  if (const char* env = std::getenv("HGX_DEBUG")) h->flags = static_cast<uint32_t>(std::atoi(env));
+  *out = h;
+  return HGX_OK;
+}
+
+void hgx_attn_destroy(hgx_attn_handle* h) {
+  if (!h) return;
+  if (h->d_lim) cudaFree(h->d_lim);
+  if (h->d_items) cudaFree(h->d_items);
+  if (h->d_err) cudaFree(h->d_err);
+  if (h->h_stage) cudaFreeHost(h->h_stage);
+  if (h->stage_done) cudaEventDestroy(h->stage_done);
+  delete h;
+}
+
+const char* hgx_attn_last_error(const hgx_attn_handle* h) {
+  return h ? h->last_error.c_str() : "null handle";
+}
+
+hgx_status hgx_attn_prologue(hgx_attn_handle* h, void* stream, void* q, void* k,
+                             const int32_t* pos_thw, const void* q_norm_w, const void* k_norm_w,
+                             int32_t total_tokens) {
+  if (!h) return HGX_ERR_INVALID_ARG;
+  h->last_error.clear();
+  if (total_tokens < 0 || total_tokens > hgx::kMaxTokens)
+    return fail(h, HGX_ERR_INVALID_ARG, "total_tokens out of range");
+  if (total_tokens == 0) return HGX_OK;
+  hgx_status st = check_tensors(h, {q, k, pos_thw, q_norm_w, k_norm_w});
+  if (st != HGX_OK) return st;
+  if ((st = ensure_device(h)) != HGX_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = hgx::launch_prologue(s, q, k, pos_thw, q_norm_w, k_norm_w, total_tokens,
+                                       h->cfg.rms_eps, h->rope);
+  if (e != cudaSuccess) return cuda_fail(h, e, "prologue launch");
+  return finish(h, s);
+}
+
+hgx_status hgx_attn_attention(hgx_attn_handle* h, void* stream, const void* q, const void* k,
+                              const void* v, void* out, int32_t batch,
+                              const int32_t* cu_seqlens_host, const hgx_segment* segs_host,
+                              const int32_t* cu_segs_host) {
+  if (!h) return HGX_ERR_INVALID_ARG;
+  h->last_error.clear();
+  std::string err;
+  int32_t T = 0;
+  hgx_status st = hgx::validate_descriptor(batch, cu_seqlens_host, segs_host, cu_segs_host,
+                                           &err, &T);
+  if (st != HGX_OK) return fail(h, st, err);
+  if (T == 0) return HGX_OK;
+  if ((st = check_tensors(h, {q, k, v, out})) != HGX_OK) return st;
+  const size_t qb = size_t(T) * 8192, kb = size_t(T) * 2048;
+  if (overlaps(out, qb, q, qb) || overlaps(out, qb, k, kb) || overlaps(out, qb, v, kb))
+    return fail(h, HGX_ERR_INVALID_ARG, "out overlaps q, k or v");
+  if ((st = ensure_device(h)) != HGX_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = prepare_plan(h, s, batch, cu_seqlens_host, segs_host, cu_segs_host)) != HGX_OK)
+    return st;
+  if ((st = run_attention(h, s, q, k, v, out)) != HGX_OK) return st;
+  return finish(h, s);
+}
+
+hgx_status hgx_attn_forward(hgx_attn_handle* h, void* stream, void* q, void* k, const void* v,
+                            void* out, const int32_t* pos_thw, const void* q_norm_w,
+                            const void* k_norm_w, int32_t batch, const int32_t* cu_seqlens_host,
+                            const hgx_segment* segs_host, const int32_t* cu_segs_host) {
+  if (!h) return HGX_ERR_INVALID_ARG;
+  h->last_error.clear();
+  std::string err;
+  int32_t T = 0;
+  hgx_status st = hgx::validate_descriptor(batch, cu_seqlens_host, segs_host, cu_segs_host,
+                                           &err, &T);
+  if (st != HGX_OK) return fail(h, st, err);
+  if (T == 0) return HGX_OK;
+  if ((st = check_tensors(h, {q, k, v, out, pos_thw, q_norm_w, k_norm_w})) != HGX_OK) return st;
+  const size_t qb = size_t(T) * 8192, kb = size_t(T) * 2048;
+  if (overlaps(out, qb, q, qb) || overlaps(out, qb, k, kb) || overlaps(out, qb, v, kb))
+    return fail(h, HGX_ERR_INVALID_ARG, "out overlaps q, k or v");
+  if ((st = ensure_device(h)) != HGX_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = prepare_plan(h, s, batch, cu_seqlens_host, segs_host, cu_segs_host)) != HGX_OK)
+    return st;
+  cudaError_t e =
+      hgx::launch_prologue(s, q, k, pos_thw, q_norm_w, k_norm_w, T, h->cfg.rms_eps, h->rope);
+  if (e != cudaSuccess) return cuda_fail(h, e, "prologue launch");
+  if ((st = run_attention(h, s, q, k, v, out)) != HGX_OK) return st;
+  return finish(h, s);
+}
+
+hgx_status hgx_attn_row_limits(int32_t batch, const int32_t* cu_seqlens_host,
+                               const hgx_segment* segs_host, const int32_t* cu_segs_host,
+                               int32_t* lim_out, size_t cap) {
+  std::vector<int32_t> lim;
+  std::string err;
+  hgx_status st = hgx::row_limits(batch, cu_seqlens_host, segs_host, cu_segs_host, &lim, &err);
+  if (st != HGX_OK) return st;
+  if (lim.empty()) return HGX_OK;
+  if (!lim_out || cap < lim.size()) return HGX_ERR_INVALID_ARG;
+  std::memcpy(lim_out, lim.data(), lim.size() * sizeof(int32_t));
+  return HGX_OK;
+}
+
+hgx_status hgx_attn_classify(int32_t batch, const int32_t* cu_seqlens_host,
+                             const hgx_segment* segs_host, const int32_t* cu_segs_host,
+                             int32_t* bm_tokens, int32_t* bn_keys, uint8_t* classes_out,
+                             size_t cap, size_t* n_written) {
+  if (bm_tokens) *bm_tokens = hgx::kBlockTokens;
+  if (bn_keys) *bn_keys = hgx::kBlockKeys;
+  hgx::Plan plan;
+  std::string err;
+  hgx_status st = hgx::build_plan(batch, cu_seqlens_host, segs_host, cu_segs_host, 1, &plan, &err);
+  if (st != HGX_OK) return st;
+  // one item per query block (a single KV head was requested); recover the block order
+  size_t total = 0;
+  for (int32_t b = 0; b < batch; ++b) {
+    const int64_t L = cu_seqlens_host[b + 1] - cu_seqlens_host[b];
+    total += static_cast<size_t>(((L + hgx::kBlockTokens - 1) / hgx::kBlockTokens) *
+                                 ((L + hgx::kBlockKeys - 1) / hgx::kBlockKeys));
+  }
+  if (n_written) *n_written = total;
+  if (!classes_out) return HGX_OK;
+  if (cap < total) return HGX_ERR_INVALID_ARG;
+  // items are sorted by cost; index them by (first token) to emit in order
+  std::vector<const hgx::WorkItem*> by_q0(static_cast<size_t>(plan.total_tokens), nullptr);
+  for (const hgx::WorkItem& it : plan.items) by_q0[static_cast<size_t>(it.q0)] = &it;
+  size_t at = 0;
+  for (int32_t b = 0; b < batch; ++b) {
+    const int32_t base = cu_seqlens_host[b];
+    const int32_t L = cu_seqlens_host[b + 1] - base;
+    const int32_t nkb = (L + hgx::kBlockKeys - 1) / hgx::kBlockKeys;
+    for (int32_t r0 = 0; r0 < L; r0 += hgx::kBlockTokens) {
+      const hgx::WorkItem* it = by_q0[static_cast<size_t>(base + r0)];
+      for (int32_t kb = 0; kb < nkb; ++kb)
+        classes_out[at++] = kb < it->n_full    ? HGX_TILE_FULL
+                            : kb < it->n_total ? HGX_TILE_PARTIAL
+                                               : HGX_TILE_SKIP;
+    }
+  }
+  return HGX_OK;
+}
+
+hgx_status hgx_attn_sync_status(hgx_attn_handle* h, void* stream) {
+  if (!h) return HGX_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(h, e, "cudaStreamSynchronize");
+  if (!h->d_err) return HGX_OK;
+  uint32_t word = 0;
+  e = cudaMemcpy(&word, h->d_err, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(h, e, "cudaMemcpy (error word)");
+  if (word) {
+    e = cudaMemset(h->d_err, 0, sizeof(uint32_t));
+    if (e != cudaSuccess) return cuda_fail(h, e, "cudaMemset (error word)");
+    char buf[128];
+    std::snprintf(buf, sizeof(buf), "a bounded device wait ran out (error word 0x%08x)", word);
+    return fail(h, HGX_ERR_TIMEOUT, buf);
+  }
+  return HGX_OK;
+}
+
+hgx_status hgx_attn_set_debug(hgx_attn_handle* h, uint32_t flags, uint64_t wait_limit_ns) {
+  if (!h) return HGX_ERR_INVALID_ARG;
+  if (flags & ~(HGX_DEBUG_CHECKED | HGX_DEBUG_STALL_TEST))
+    return fail(h, HGX_ERR_INVALID_ARG, "unknown debug flag");
+  h->flags = flags;
+  h->wait_limit_ns = wait_limit_ns ? wait_limit_ns : 2000000000ull;
+  return HGX_OK;
+}
+
+}  // extern "C"

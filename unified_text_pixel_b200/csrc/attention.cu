@@ -1,0 +1,463 @@
+// Masked GQA flash attention for sm_100a: TMA-fed K/V staging, tcgen05 MMAs accumulating
+// in tensor memory, per-row online softmax, GQA head packing and per-tile mask skipping.
+//
+// What it computes (sources named by page title and section):
+//   out[i, h] = sum_{j < lim(i)} softmax_j(q'[i,h] . k'[j,h/4] * scale) v[j,h/4]
+// with 32 query heads over 8 KV heads at head_dim 128 ("hidream-o1-p100a" model card, "What
+// this model is"), and lim(i) the exclusive key limit that the HiDream-O1 mask (model card,
+// "What this model is"; "HiDream-O1-Image" summary, "How it works") or the HunyuanImage 3.0
+// Generalized Causal Attention (paper-graph-ui summary, section 3.4, "The core rule")
+// gives row i. Every visible set is a prefix of the keys, so a tile of (query block, key
+// block) is either fully visible, fully masked (skipped: no MMA is issued) or needs one
+// integer compare per score.
+//
+// CTA organisation (one CTA per SM, persistent over a longest-first work list):
+//   work item = one KV head g, its 4 query heads, 64 consecutive query tokens.
+//   The item is two MMA tiles of M = 128 rows; row r of tile X is token
+//   q0 + 32 X + r / 4 and query head 4 g + r % 4, so every K/V tile staged in shared
+//   memory serves all 4 query heads of its KV head (GQA sharing) and both tiles.
+//   warp 0      TMA producer: Q tiles, then K_j, V_j into a 4-slot ring (32 KB per slot)
+//   warp 1      TMEM allocator and the single-thread tcgen05.mma issuer
+//   warps 4-7   softmax of tile 0, warps 8-11 softmax of tile 1 (one thread per row)
+// Tensor memory (512 columns): S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512);
+// P (bf16) is written over the first 64 columns of its S and read by the PV MMA from
+// tensor memory. The MMA warp interleaves the tiles so that one tile's softmax runs while
+// the tensor core works on the other's QK^T and PV:
+//   S0(0) S1(0) | PV0(j-1) S0(j) PV1(j-1) S1(j) | ... | PV0(n-1) PV1(n-1)
+// Online softmax keeps the running maximum that was last used for exponentiation and only
+// rescales O (in tensor memory) and the row sum when the maximum grows by more than 2^8,
+// so probabilities stay below 256 and O is rarely touched.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace hgx {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 384;
+constexpr int kStages = 4;                    // K/V ring slots
+constexpr uint32_t kTileBytes = 32768;        // 128 rows x 128 bf16
+constexpr uint32_t kHalfBytes = 16384;        // 128 rows x 64 bf16 (one 128-byte swizzle span)
+constexpr uint32_t kQBytes = 2 * kTileBytes;  // both Q tiles of an item
+constexpr uint32_t kRingOffset = kQBytes;
+constexpr uint32_t kBarOffset = kRingOffset + kStages * kTileBytes;
+// barrier slots (8 bytes each)
+enum : uint32_t {
+  BAR_Q_FULL = 0,
+  BAR_Q_EMPTY = 1,
+  BAR_KV_FULL = 2,                   // + slot
+  BAR_KV_EMPTY = BAR_KV_FULL + kStages,
+  BAR_S_FULL = BAR_KV_EMPTY + kStages,  // + tile
+  BAR_P_FULL = BAR_S_FULL + 2,
+  BAR_O_FULL = BAR_P_FULL + 2,
+  BAR_O_EMPTY = BAR_O_FULL + 2,
+  BAR_STALL = BAR_O_EMPTY + 2,       // debug: nothing ever arrives here
+  BAR_DRAIN = BAR_STALL + 1,
+  BAR_COUNT = BAR_DRAIN + 1
+};
+constexpr uint32_t kMiscOffset = kBarOffset + 8 * BAR_COUNT;  // tmem base, abort flag
+constexpr uint32_t kSmemUsed = kMiscOffset + 16;
+constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // slack to align the base to 1024 B
+
+constexpr uint32_t kTmemCols = 512;
+__host__ __device__ constexpr uint32_t col_s(int x) { return 128u * x; }        // S0, S1
+__host__ __device__ constexpr uint32_t col_o(int x) { return 256u + 128u * x; } // O0, O1
+
+constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, false);  // S = Q K^T, both K-major
+constexpr uint32_t kIdescPV = idesc_bf16_f32(128, 128, true);   // O += P V, V N-major
+
+// error sites (bits 8..15 of the error word) to tell which wait ran out
+enum : uint32_t {
+  SITE_PRODUCER = 1,
+  SITE_MMA = 2,
+  SITE_SOFTMAX = 3,
+  SITE_STALL = 4,
+  SITE_DRAIN = 5
+};
+
+struct Ctx {
+  uint32_t bars;           // shared address of barrier 0
+  volatile uint32_t* abort_flag;
+  uint32_t* err;
+  uint64_t limit_ns;
+};
+
+__device__ __forceinline__ uint32_t bar_addr(const Ctx& c, uint32_t i) { return c.bars + 8 * i; }
+
+// Bounded wait for the phase of the given parity. Returns false if the wait ran out (after
+// recording it in the device error word and raising the CTA's abort flag) or if another
+// role already raised the abort flag.
+__device__ __noinline__ bool wait_bounded(const Ctx& c, uint32_t bar, uint32_t parity,
+                                          uint32_t site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  uint64_t start = 0;
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*c.abort_flag) return false;
+    if ((it & 63u) == 0) {
+      const uint64_t now = globaltimer_ns();
+      if (start == 0) {
+        start = now;
+      } else if (now - start > c.limit_ns) {
+        *c.abort_flag = 1u;
+        atomicOr(c.err, kErrTimeout | (site << 8));
+        return false;
+      }
+    }
+  }
+}
+
+// Bounded wait that ignores the abort flag: used while draining copies and MMAs that are
+// already in flight, which complete on their own.
+__device__ __noinline__ void wait_drain(const Ctx& c, uint32_t bar, uint32_t parity) {
+  const uint64_t start = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - start > c.limit_ns) {
+      atomicOr(c.err, kErrTimeout | (SITE_DRAIN << 8));
+      return;
+    }
+  }
+}
+
+// S_X = Q_X K^T over head_dim 128: 8 MMAs of K = 16. Both operands K-major with 128-byte
+// swizzle: rows of 128 B (64 features), 8-row groups 1024 B apart (SBO); features 64..127
+// sit in the second 16 KB half of the tile.
+__device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint32_t q_tile, uint32_t k_tile) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+    const uint64_t a = smem_desc_sw128(q_tile + off, 16, 1024);
+    const uint64_t b = smem_desc_sw128(k_tile + off, 16, 1024);
+    mma_ss(tmem_s, a, b, kIdescQK, kk > 0 ? 1u : 0u);
+  }
+}
+
+// O_X (+)= P_X V: 8 MMAs of K = 16 keys. P (bf16, 2 per column) is read from tensor
+// memory; V is [keys, head_dim] with head_dim contiguous (N-major for the B operand):
+// 8-key groups 1024 B apart (SBO), the two 64-feature halves 16 KB apart (LBO).
+__device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_tile,
+                                         bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint64_t b = smem_desc_sw128(v_tile + kk * 2048, kHalfBytes, 1024);
+    mma_ts(tmem_o, tmem_p + kk * 8, b, kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attention_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                     const __grid_constant__ CUtensorMap tmap_k,
+                     const __grid_constant__ CUtensorMap tmap_v, const AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;  // 128-byte swizzle wants 1024-B alignment
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t sQ = base;
+  const uint32_t sRing = base + kRingOffset;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(gbase + kMiscOffset);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(gbase + kMiscOffset + 4);
+  Ctx c{base + kBarOffset, abort_flag, p.err, p.wait_limit_ns};
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_addr(c, BAR_Q_FULL), 1);
+    mbar_init(bar_addr(c, BAR_Q_EMPTY), 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bar_addr(c, BAR_KV_FULL + s), 1);
+      mbar_init(bar_addr(c, BAR_KV_EMPTY + s), 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bar_addr(c, BAR_S_FULL + x), 1);
+      mbar_init(bar_addr(c, BAR_P_FULL + x), 128);
+      mbar_init(bar_addr(c, BAR_O_FULL + x), 1);
+      mbar_init(bar_addr(c, BAR_O_EMPTY + x), 128);
+    }
+    mbar_init(bar_addr(c, BAR_STALL), 1);
+    mbar_init(bar_addr(c, BAR_DRAIN), 1);
+    *abort_flag = 0u;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_holder)), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmap_q);
+      tma_prefetch_desc(&tmap_k);
+      tma_prefetch_desc(&tmap_v);
+      uint32_t pos = 0, qe_par = 0, q_loads = 0;
+      int32_t last_round[kStages];
+      for (int s = 0; s < kStages; ++s) last_round[s] = -1;
+      bool ok = true;
+      for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
+        const WorkItem it = p.items[w];
+        if (q_loads > 0) {
+          ok = wait_bounded(c, bar_addr(c, BAR_Q_EMPTY), qe_par, SITE_PRODUCER);
+          qe_par ^= 1u;
+          if (!ok) break;
+        }
+        mbar_arrive_expect_tx(bar_addr(c, BAR_Q_FULL), kQBytes);
+        for (int x = 0; x < 2; ++x) {
+          // a tile that starts past the last token only holds rows that are never stored:
+          // start it at the last token so that no box lies wholly outside the tensor
+          const int32_t t0 = min(it.q0 + 32 * x, p.total_tokens - 1);
+          for (int hf = 0; hf < 2; ++hf)
+            tma_load_3d(sQ + x * kTileBytes + hf * kHalfBytes, &tmap_q, bar_addr(c, BAR_Q_FULL),
+                        64 * hf, 4 * it.g, t0);
+        }
+        ++q_loads;
+        for (int j = 0; ok && j < it.n_total; ++j) {
+          for (int kv = 0; kv < 2; ++kv) {  // K_j then V_j
+            const uint32_t slot = pos % kStages;
+            const uint32_t round = pos / kStages;
+            ok = wait_bounded(c, bar_addr(c, BAR_KV_EMPTY + slot), (round & 1u) ^ 1u,
+                              SITE_PRODUCER);
+            if (!ok) break;
+            const uint32_t full = bar_addr(c, BAR_KV_FULL + slot);
+            mbar_arrive_expect_tx(full, kTileBytes);
+            const CUtensorMap* map = kv == 0 ? &tmap_k : &tmap_v;
+            for (int hf = 0; hf < 2; ++hf)
+              tma_load_3d(sRing + slot * kTileBytes + hf * kHalfBytes, map, full, 64 * hf, it.g,
+                          it.kv0 + 128 * j);
+            last_round[slot] = static_cast<int32_t>(round);
+            ++pos;
+          }
+        }
+      }
+      // drain: every load this thread issued must land before the CTA exits (on the normal
+      // path they all have, and these waits return at once)
+      for (int s = 0; s < kStages; ++s)
+        if (last_round[s] >= 0)
+          wait_drain(c, bar_addr(c, BAR_KV_FULL + s), static_cast<uint32_t>(last_round[s]) & 1u);
+      if (q_loads > 0) wait_drain(c, bar_addr(c, BAR_Q_FULL), (q_loads - 1) & 1u);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t pos = 0, qf_par = 0;
+      uint32_t p_par[2] = {0, 0}, oe_par[2] = {0, 0};
+      bool first = true, ok = true;
+      auto wait_kv = [&](uint32_t ps) {
+        return wait_bounded(c, bar_addr(c, BAR_KV_FULL + ps % kStages), (ps / kStages) & 1u,
+                            SITE_MMA);
+      };
+      auto slot_addr = [&](uint32_t ps) { return sRing + (ps % kStages) * kTileBytes; };
+      auto release = [&](uint32_t ps) { mma_commit(bar_addr(c, BAR_KV_EMPTY + ps % kStages)); };
+      // wait until softmax X has written P (and rescaled O); before the first PV of an item
+      // also wait until the previous item's epilogue has read O
+      auto wait_p = [&](int x, bool first_pv) {
+        if (!wait_bounded(c, bar_addr(c, BAR_P_FULL + x), p_par[x], SITE_MMA)) return false;
+        p_par[x] ^= 1u;
+        if (first_pv && !first) {
+          if (!wait_bounded(c, bar_addr(c, BAR_O_EMPTY + x), oe_par[x], SITE_MMA)) return false;
+          oe_par[x] ^= 1u;
+        }
+        tc_fence_after();
+        return true;
+      };
+      for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
+        const WorkItem it = p.items[w];
+        const int n = it.n_total;
+        if (!(ok = wait_bounded(c, bar_addr(c, BAR_Q_FULL), qf_par, SITE_MMA))) break;
+        qf_par ^= 1u;
+        uint32_t kpos = pos++;
+        if (!(ok = wait_kv(kpos))) break;
+        tc_fence_after();
+        issue_qk(tmem + col_s(0), sQ, slot_addr(kpos));
+        mma_commit(bar_addr(c, BAR_S_FULL + 0));
+        issue_qk(tmem + col_s(1), sQ + kTileBytes, slot_addr(kpos));
+        mma_commit(bar_addr(c, BAR_S_FULL + 1));
+        if (n == 1) mma_commit(bar_addr(c, BAR_Q_EMPTY));
+        release(kpos);
+        for (int j = 1; j < n; ++j) {
+          const uint32_t vpos = pos++;
+          kpos = pos++;
+          if (!(ok = wait_kv(vpos) && wait_kv(kpos))) break;
+          if (!(ok = wait_p(0, j == 1))) break;
+          issue_pv(tmem + col_o(0), tmem + col_s(0), slot_addr(vpos), j > 1);
+          issue_qk(tmem + col_s(0), sQ, slot_addr(kpos));
+          mma_commit(bar_addr(c, BAR_S_FULL + 0));
+          if (!(ok = wait_p(1, j == 1))) break;
+          issue_pv(tmem + col_o(1), tmem + col_s(1), slot_addr(vpos), j > 1);
+          release(vpos);
+          issue_qk(tmem + col_s(1), sQ + kTileBytes, slot_addr(kpos));
+          mma_commit(bar_addr(c, BAR_S_FULL + 1));
+          if (j == n - 1) mma_commit(bar_addr(c, BAR_Q_EMPTY));
+          release(kpos);
+        }
+        if (!ok) break;
+        const uint32_t vpos = pos++;
+        if (!(ok = wait_kv(vpos))) break;
+        if (!(ok = wait_p(0, n == 1))) break;
+        issue_pv(tmem + col_o(0), tmem + col_s(0), slot_addr(vpos), n > 1);
+        mma_commit(bar_addr(c, BAR_O_FULL + 0));
+        if (!(ok = wait_p(1, n == 1))) break;
+        issue_pv(tmem + col_o(1), tmem + col_s(1), slot_addr(vpos), n > 1);
+        mma_commit(bar_addr(c, BAR_O_FULL + 1));
+        release(vpos);
+        first = false;
+      }
+      // every MMA this thread issued must complete before tensor memory is freed
+      mma_commit(bar_addr(c, BAR_DRAIN));
+      wait_drain(c, bar_addr(c, BAR_DRAIN), 0);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------------ softmax
+    const int x = (warp - 4) >> 2;      // tile
+    const int quarter = warp & 3;       // tensor-memory lanes 32*quarter .. +31
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_bits = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_bits + col_s(x);
+    const uint32_t tO = tmem + lane_bits + col_o(x);
+    const float sl2 = p.scale_log2;
+    uint32_t s_par = 0, o_par = 0;
+    bool ok = true;
+    if ((p.flags & HGX_DEBUG_STALL_TEST) && x == 0)
+      ok = __all_sync(0xffffffffu, wait_bounded(c, bar_addr(c, BAR_STALL), 0, SITE_STALL));
+    for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
+      const WorkItem it = p.items[w];
+      const int32_t tok = it.q0 + 32 * x + (row >> 2);
+      const int32_t head = 4 * it.g + (row & 3);
+      const bool valid = tok - it.kv0 < it.len;
+      const int32_t row_lim = valid ? p.lim[tok] : it.len;
+      float m_used = -INFINITY, l = 0.f;
+      for (int j = 0; j < it.n_total; ++j) {
+        ok = __all_sync(0xffffffffu, wait_bounded(c, bar_addr(c, BAR_S_FULL + x), s_par,
+                                                   SITE_SOFTMAX));
+        if (!ok) break;
+        s_par ^= 1u;
+        tc_fence_after();
+        uint32_t sr[4][32];
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) tmem_ld32(tS + 32 * ch, sr[ch]);
+        tmem_wait_ld();
+        float s[128];
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) s[32 * ch + e] = __uint_as_float(sr[ch][e]);
+        if (j >= it.n_full) {
+          const int nvis = row_lim - 128 * j;  // keys [0, nvis) of this block are visible
+#pragma unroll
+          for (int e = 0; e < 128; ++e)
+            if (e >= nvis) s[e] = -INFINITY;
+        }
+        float mx = s[0];
+#pragma unroll
+        for (int e = 1; e < 128; ++e) mx = fmaxf(mx, s[e]);
+        const float m_new = fmaxf(m_used, mx);
+        if (j == 0) {
+          m_used = m_new;
+        } else if ((m_new - m_used) * sl2 > 8.0f) {
+          const float alpha = ex2_approx((m_used - m_new) * sl2);
+          l *= alpha;
+          m_used = m_new;
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * ch, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(tO + 32 * ch, o);
+          }
+        }
+        const float mb = m_used * sl2;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {  // 32 keys -> 16 packed columns at a time
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = ex2_approx(fmaf(s[32 * q4 + 2 * e], sl2, -mb));
+            const float p1 = ex2_approx(fmaf(s[32 * q4 + 2 * e + 1], sl2, -mb));
+            l += p0 + p1;
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(tS + 16 * q4, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar_addr(c, BAR_P_FULL + x));
+      }
+      if (!ok) break;
+      // epilogue: O / l -> bf16 -> out[tok, head, :]
+      ok = __all_sync(0xffffffffu, wait_bounded(c, bar_addr(c, BAR_O_FULL + x), o_par,
+                                                 SITE_SOFTMAX));
+      if (!ok) break;
+      o_par ^= 1u;
+      tc_fence_after();
+      const float inv_l = 1.0f / l;
+      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) +
+                           (static_cast<size_t>(tok) * 32 + head) * 128;
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t o[32];
+        tmem_ld32(tO + 32 * ch, o);
+        tmem_wait_ld();
+        if (valid) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l,
+                                __uint_as_float(o[2 * e + 1]) * inv_l);
+          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * ch);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            d4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar_addr(c, BAR_O_EMPTY + x));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+size_t attention_smem_bytes() { return kSmemBytes; }
+
+cudaError_t launch_attention(cudaStream_t stream, const CUtensorMap& tmap_q,
+                             const CUtensorMap& tmap_k, const CUtensorMap& tmap_v,
+                             const AttnParams& p, int grid) {
+  static uint64_t configured = 0;  // bit per device: shared-memory limit raised
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 64 || !(configured & (1ull << dev))) {
+    e = cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes));
+    if (e != cudaSuccess) return e;
+    if (dev < 64) configured |= 1ull << dev;
+  }
+  attention_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tmap_q, tmap_k, tmap_v, p);
+  return cudaGetLastError();
+}
+
+}  // namespace hgx

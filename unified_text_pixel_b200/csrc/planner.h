@@ -1,0 +1,64 @@
+// Host planner of the hybrid-masked attention: descriptor validation, per-row key limits,
+// tile classes and the attention kernel's work list. Pure C++ (no CUDA calls), so every
+// part of it runs and is tested on a machine without a GPU.
+#pragma once
+
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include "../../include/hgx_attn.h"
+
+namespace hgx {
+
+// Tile of the attention kernel: kBlockTokens query tokens (x 4 query heads of one KV head,
+// as two 128-row MMA tiles of 32 tokens each) against kBlockKeys keys.
+constexpr int kTileTokens = 32;                 // tokens per 128-row MMA tile (4 heads each)
+constexpr int kTilesPerBlock = 2;               // MMA tiles per work item (ping-pong)
+constexpr int kBlockTokens = kTileTokens * kTilesPerBlock;
+constexpr int kBlockKeys = 128;
+// Largest packed token count: keeps every byte offset of q/out (T * 8192) below 2^32 and
+// every TMA coordinate far inside int32.
+constexpr int32_t kMaxTokens = (1 << 19) - 1;
+
+// One unit of attention work: one KV head g and its 4 query heads over kBlockTokens
+// consecutive query tokens of one batch element. Layout shared with the kernel.
+struct WorkItem {
+  int32_t q0;       // packed index of the first query token
+  int32_t kv0;      // packed index of the batch element's first token
+  int32_t len;      // tokens in the batch element
+  int32_t g;        // KV head
+  int32_t n_full;   // key blocks [0, n_full) are visible to every row: no mask compare
+  int32_t n_total;  // key blocks [n_full, n_total) need the per-row compare; the rest skip
+  int32_t pad0, pad1;
+};
+static_assert(sizeof(WorkItem) == 32, "work item layout");
+
+struct Plan {
+  int32_t batch = 0;
+  int32_t total_tokens = 0;
+  std::vector<int32_t> lim;        // [T] exclusive key limit per packed row, local
+  std::vector<WorkItem> items;     // sorted by n_total, longest first
+  uint64_t visible_pairs = 0;      // sum of lim over all rows
+};
+
+// Checks the packed-varlen descriptor. On failure returns INVALID_ARG with *err set.
+hgx_status validate_descriptor(int32_t batch, const int32_t* cu_seqlens,
+                               const hgx_segment* segs, const int32_t* cu_segs,
+                               std::string* err, int32_t* total_tokens);
+
+// Validates and fills lim (size T). Returns INVALID_ARG on a bad descriptor.
+hgx_status row_limits(int32_t batch, const int32_t* cu_seqlens, const hgx_segment* segs,
+                      const int32_t* cu_segs, std::vector<int32_t>* lim, std::string* err);
+
+// Validates, computes limits and the sorted work list for num_kv_heads KV heads.
+hgx_status build_plan(int32_t batch, const int32_t* cu_seqlens, const hgx_segment* segs,
+                      const int32_t* cu_segs, int32_t num_kv_heads, Plan* plan,
+                      std::string* err);
+
+// Frequency table of the interleaved mRoPE: inv_freq[k] = theta^(-2k/D) and the axis
+// (0 t, 1 h, 2 w) that drives frequency k.
+void mrope_tables(double theta, int32_t head_dim, const int32_t section[3], double* inv_freq,
+                  int32_t* axis);
+
+}  // namespace hgx

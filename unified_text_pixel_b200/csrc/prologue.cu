@@ -1,0 +1,124 @@
+// Prologue: q/k RMSNorm and interleaved 3-axis mRoPE, in place, bf16 in and out.
+//
+// "hidream-o1-p100a" model card, "What this model is": the language model applies "q/k
+// RMSNorm" and "3-axis interleaved mRoPE [24,20,20] at theta 5e6" (32 query heads, 8 KV
+// heads, head 128). Rotation pairs feature k with feature k + 64, the half-split layout of
+// the 1D RoPE definition in "HunyuanImage 3.0 Technical Report" (paper-graph-ui summary),
+// section 3.4, "Generalized 2D Rotary Position Embedding (RoPE)".
+//
+// Layout: one block handles kTok tokens and all 40 heads (32 q + 8 k) of each. A head's
+// 128 bf16 (256 B) is read by a half-warp as 16-byte loads, so a warp reads 512
+// contiguous bytes; lanes j and j + 8 of a half-warp hold the partners (k, k + 64) of a
+// rotation and swap values with one shuffle. Angles are computed once per (token, k) in
+// fp64 (positions reach ~10^4 rad, far outside the range where a float angle keeps
+// precision) and shared by all 40 heads through shared memory. HBM-bound: every byte of
+// q and k is read once and written once.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "kernels.h"
+
+namespace hgx {
+
+namespace {
+
+constexpr int kTok = 4;          // tokens per block
+constexpr int kThreads = 256;    // 16 half-warps: 16 heads in flight
+constexpr int kHeads = 40;       // 32 query + 8 key heads per token
+constexpr int kHalf = 64;        // rotation pairs per head
+
+__device__ __forceinline__ void unpack8(const uint4& r, float (&x)[8]) {
+  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&y)[8]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __nv_bfloat162 b = __floats2bfloat162_rn(y[2 * i], y[2 * i + 1]);
+    w[i] = *reinterpret_cast<uint32_t*>(&b);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+__global__ void __launch_bounds__(kThreads) prologue_kernel(
+    __nv_bfloat16* __restrict__ q, __nv_bfloat16* __restrict__ k,
+    const int32_t* __restrict__ pos, const __nv_bfloat16* __restrict__ wq,
+    const __nv_bfloat16* __restrict__ wk, int32_t T, float eps, const RopeTables tab) {
+  __shared__ float2 cs[kTok][kHalf];  // (cos, sin) per token and frequency
+  const int t0 = blockIdx.x * kTok;
+  {
+    const int tl = threadIdx.x / kHalf;
+    const int f = threadIdx.x % kHalf;
+    const int t = t0 + tl;
+    float c = 1.f, s = 0.f;
+    if (t < T) {
+      const double phi = static_cast<double>(pos[3 * t + tab.axis[f]]) * tab.inv_freq[f];
+      double sd, cd;
+      sincos(phi, &sd, &cd);
+      c = static_cast<float>(cd);
+      s = static_cast<float>(sd);
+    }
+    cs[tl][f] = make_float2(c, s);
+  }
+  const int j = threadIdx.x & 15;  // 16-byte chunk of the head: features 8j .. 8j+7
+  float wqv[8], wkv[8];
+  unpack8(*reinterpret_cast<const uint4*>(wq + 8 * j), wqv);
+  unpack8(*reinterpret_cast<const uint4*>(wk + 8 * j), wkv);
+  __syncthreads();
+
+  const bool low = j < 8;          // features < 64: first member of each pair
+  const int f0 = (j & 7) * 8;      // frequency of this lane's first feature
+  for (int u = threadIdx.x >> 4; u < kTok * kHeads; u += kThreads / 16) {
+    const int tl = u / kHeads;
+    const int hh = u % kHeads;
+    const int t = t0 + tl;
+    const bool valid = t < T;
+    __nv_bfloat16* base = hh < 32 ? q + (static_cast<size_t>(t) * 32 + hh) * 128
+                                  : k + (static_cast<size_t>(t) * 8 + (hh - 32)) * 128;
+    float x[8];
+    uint4 raw = make_uint4(0, 0, 0, 0);
+    if (valid) raw = *reinterpret_cast<const uint4*>(base + 8 * j);
+    unpack8(raw, x);
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
+#pragma unroll
+    for (int off = 8; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    const float r = rsqrtf(ss * (1.f / 128.f) + eps);
+    const float* w = hh < 32 ? wqv : wkv;
+    float y[8], yp[8], o[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) y[e] = x[e] * r * w[e];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) yp[e] = __shfl_xor_sync(0xffffffffu, y[e], 8);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float2 c = cs[tl][f0 + e];
+      o[e] = low ? fmaf(y[e], c.x, -yp[e] * c.y) : fmaf(y[e], c.x, yp[e] * c.y);
+    }
+    if (valid) *reinterpret_cast<uint4*>(base + 8 * j) = pack8(o);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_prologue(cudaStream_t stream, void* q, void* k, const int32_t* pos,
+                            const void* wq, const void* wk, int32_t T, float eps,
+                            const RopeTables& tab) {
+  if (T <= 0) return cudaSuccess;
+  const int grid = (T + kTok - 1) / kTok;
+  prologue_kernel<<<grid, kThreads, 0, stream>>>(
+      static_cast<__nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(k), pos,
+      static_cast<const __nv_bfloat16*>(wq), static_cast<const __nv_bfloat16*>(wk), T, eps, tab);
+  return cudaGetLastError();
+}
+
+}  // namespace hgx

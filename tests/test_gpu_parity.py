@@ -140,6 +140,39 @@ def test_attention_alone_on_kernel_rotated_inputs(hgx):
         assert err.max() <= 1e-2 and err.mean() <= 5e-4, (float(err.max()), float(err.mean()))
 
 
+def test_online_rescale_path_with_divergent_rows(hgx):
+    """Key norms that grow along the sequence make the running row maximum jump by far
+    more than 2^8 (in exp2 units) from one key block to the next, differently for every
+    row, so the kernel's O/row-sum rescaling runs for some rows of a warp and not for
+    others. Attention alone on given bf16 q'/k' against the oracle's masked softmax."""
+    H, a = hgx
+    w = W.custom("ramp", [[(300, W.CAUSAL), (400, W.FULL_SEQUENCE)], [(200, W.FULL_IN_SEGMENT), (333, W.CAUSAL)]],
+                 seed=31)
+    T = w.total_tokens
+    g = torch.Generator().manual_seed(31)
+    q = torch.randn(T, 32, 128, generator=g)
+    k = torch.randn(T, 8, 128, generator=g)
+    v = torch.randn(T, 8, 128, generator=g)
+    # per batch element, key norms grow 120-fold from its first to its last token
+    ramp = torch.cat([0.1 + 12.0 * torch.linspace(0, 1, L) ** 2 for L in w.lengths])
+    k = k * ramp[:, None, None]
+    q[:, ::3] *= 0.1  # some heads stay flat: rows of one warp disagree on rescaling
+    qb, kb, vb = (x.to(torch.bfloat16) for x in (q, k, v))
+    out = torch.empty(T, 32, 128, dtype=torch.bfloat16, device="cuda")
+    a.attention(qb.cuda(), kb.cuda(), vb.cuda(), out, *_desc(w))
+    assert a.sync_status() == H.HGX_OK
+    cu, segs, cu_segs = _desc(w)
+    got = out.float().cpu().numpy()
+    f64 = lambda x: x.float().numpy().astype(np.float64)
+    for b in range(len(cu) - 1):
+        t0, t1 = int(cu[b]), int(cu[b + 1])
+        bsegs = [tuple(int(x) for x in segs[n]) for n in range(cu_segs[b], cu_segs[b + 1])]
+        ref = O.masked_gqa_attention(f64(qb[t0:t1]), f64(kb[t0:t1]), f64(vb[t0:t1]), O.dense_mask(bsegs, t1 - t0))
+        err = np.abs(got[t0:t1] - ref)
+        assert np.isfinite(got[t0:t1]).all()
+        assert err.max() <= ATOL_MAX and err.mean() <= ATOL_MEAN, (float(err.max()), float(err.mean()))
+
+
 def test_single_token_returns_its_value(hgx):
     """One causal token sees only itself: out[0, h] == v[0, h // 4] (rounded to bf16)."""
     w = W.custom("one", [[(1, W.CAUSAL)]], seed=5)

@@ -368,7 +368,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float m_new = fmaxf(m_used, mx);
         if (j == 0) {
           m_used = m_new;
-        } else if ((m_new - m_used) * sl2 > 8.0f) {
+        } else if (__any_sync(0xffffffffu, (m_new - m_used) * sl2 > 8.0f)) {
+          // warp-uniform: the tensor-memory loads and stores below are warp-collective, so
+          // when any row of the warp needs it, every row rescales (by its own factor <= 1)
           const float alpha = ex2_approx((m_used - m_new) * sl2);
           l *= alpha;
           m_used = m_new;

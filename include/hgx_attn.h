@@ -178,6 +178,36 @@ hgx_status hgx_attn_sync_status(hgx_attn_handle* h, void* stream);
  * flags of new handles. */
 hgx_status hgx_attn_set_debug(hgx_attn_handle* h, uint32_t flags, uint64_t wait_limit_ns);
 
+/* ---------------------------------------------------------------------------------------
+ * Allocation-free variant of hgx_attn_forward. The paper has no counterpart to this entry
+ * point; it exists for callers that cannot allocate memory: code inside a framework that
+ * owns all device memory through its own pool and forbids cudaMalloc behind its back, or a
+ * process whose device footprint must not grow after start-up. It needs no handle (creating
+ * one allocates) and calls no cudaMalloc, cudaFree, cudaMallocHost or heap allocation.
+ *
+ * Scratch (per-row key limits, work list, error word) lives in one fixed-size device array
+ * inside the library (about 145 KB, held by every GPU that loads the library until the
+ * process exits); planning uses fixed-size static host buffers. Hence the limits:
+ * at most HGX_NOALLOC_MAX_TOKENS packed tokens and HGX_NOALLOC_MAX_BATCH batch elements;
+ * larger requests return HGX_ERR_UNSUPPORTED before any device work.
+ *
+ * Arguments are those of hgx_attn_forward with the config in place of a handle (validated
+ * on every call), plus `synchronize`: when nonzero the call waits for the stream and returns
+ * HGX_ERR_TIMEOUT if a bounded device wait ran out; when zero it returns after the launches
+ * and such a timeout goes unreported. The first call on each device looks up the device
+ * address of the scratch array (cudaGetSymbolAddress, with that device current); make that
+ * first call before any stream capture. All calls share the scratch and the host buffers,
+ * which keep the previous call's contents (the error word is cleared at the start of each
+ * call): calls that overlap on the GPU, or run from several host threads at once, race. */
+#define HGX_NOALLOC_MAX_TOKENS 16384
+#define HGX_NOALLOC_MAX_BATCH 64
+
+hgx_status hgx_attn_forward_noalloc(const hgx_attn_config* cfg, void* stream, void* q, void* k,
+                                    const void* v, void* out, const int32_t* pos_thw,
+                                    const void* q_norm_w, const void* k_norm_w, int32_t batch,
+                                    const int32_t* cu_seqlens_host, const hgx_segment* segs_host,
+                                    const int32_t* cu_segs_host, int32_t synchronize);
+
 #ifdef __cplusplus
 }
 #endif

@@ -32,6 +32,7 @@
 
 #include <cstdint>
 
+#include "exp2_poly.h"
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -94,29 +95,34 @@ __device__ __forceinline__ uint32_t bar_addr(const Ctx& c, uint32_t i) { return 
 // Bounded wait for the phase of the given parity. Returns false if the wait ran out (after
 // recording it in the device error word and raising the CTA's abort flag) or if another
 // role already raised the abort flag.
-__device__ __noinline__ bool wait_bounded(const Ctx& c, uint32_t bar, uint32_t parity,
-                                          uint32_t site) {
-  if (mbar_try_wait(bar, parity)) return true;
+__device__ __forceinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
+                                       uint32_t* err, uint64_t limit_ns, uint32_t site) {
   uint64_t start = 0;
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*c.abort_flag) return false;
+    if (*abort_flag) return false;
     if ((it & 63u) == 0) {
       const uint64_t now = globaltimer_ns();
       if (start == 0) {
         start = now;
-      } else if (now - start > c.limit_ns) {
-        *c.abort_flag = 1u;
-        atomicOr(c.err, kErrTimeout | (site << 8));
+      } else if (now - start > limit_ns) {
+        *abort_flag = 1u;
+        atomicOr(err, kErrTimeout | (site << 8));
         return false;
       }
     }
   }
 }
 
+__device__ __forceinline__ bool wait_bounded(const Ctx& c, uint32_t bar, uint32_t parity,
+                                             uint32_t site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return wait_slow(bar, parity, c.abort_flag, c.err, c.limit_ns, site);
+}
+
 // Bounded wait that ignores the abort flag: used while draining copies and MMAs that are
 // already in flight, which complete on their own.
-__device__ __noinline__ void wait_drain(const Ctx& c, uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ void wait_drain(const Ctx& c, uint32_t bar, uint32_t parity) {
   const uint64_t start = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
     if (globaltimer_ns() - start > c.limit_ns) {
@@ -149,6 +155,48 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint3
     const uint64_t b = smem_desc_sw128(v_tile + kk * 2048, kHalfBytes, 1024);
     mma_ts(tmem_o, tmem_p + kk * 8, b, kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
   }
+}
+
+#ifndef HGX_EXP_POLY_EVERY
+// One key pair in this many takes the FMA-pipe polynomial exp2 instead of the MUFU ex2;
+// 0 = never. Measured on B200 (edit step): the softmax is limited by instruction issue,
+// not by the MUFU, and every fraction tried (1/8, 1/4, 1/2) was slower than none.
+#define HGX_EXP_POLY_EVERY 0
+#endif
+
+// p = 2^(s * scale_log2 - mb) for the row's 128 scores, packed to bf16 pairs and stored as
+// P over the first 64 columns of S (key 2c in the low half of column c). Scale-and-shift
+// and the row sum run as paired fp32 instructions; the row sum is kept in 4 partial sums
+// (two pairs) returned in l4.
+template <bool kPoly>
+__device__ __forceinline__ void exp_store_p(const float (&s)[128], float sl2, float mb,
+                                            uint32_t tS, float (&l4)[4]) {
+  const uint64_t scale2 = f2_pack(sl2, sl2);
+  const uint64_t shift2 = f2_pack(-mb, -mb);
+  uint64_t acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {  // 32 keys -> 16 packed columns at a time
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      float x0, x1;
+      f2_unpack(ffma2(f2_pack(s[32 * q4 + 2 * e], s[32 * q4 + 2 * e + 1]), scale2, shift2), x0, x1);
+      float p0, p1;
+      if (kPoly && HGX_EXP_POLY_EVERY > 0 &&
+          (e % (HGX_EXP_POLY_EVERY > 0 ? HGX_EXP_POLY_EVERY : 1)) == HGX_EXP_POLY_EVERY - 1) {
+        p0 = exp2_poly3(x0);
+        p1 = exp2_poly3(x1);
+      } else {
+        p0 = ex2_approx(x0);
+        p1 = ex2_approx(x1);
+      }
+      acc[e & 1] = fadd2(acc[e & 1], f2_pack(p0, p1));
+      pk[e] = pack_bf16x2(p0, p1);
+    }
+    tmem_st16(tS + 16 * q4, pk);
+  }
+  f2_unpack(acc[0], l4[0], l4[1]);
+  f2_unpack(acc[1], l4[2], l4[3]);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -197,131 +245,149 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tmap_q);
-      tma_prefetch_desc(&tmap_k);
-      tma_prefetch_desc(&tmap_v);
-      uint32_t pos = 0, qe_par = 0, q_loads = 0;
-      int32_t last_round[kStages];
-      for (int s = 0; s < kStages; ++s) last_round[s] = -1;
-      bool ok = true;
-      for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
-        const WorkItem it = p.items[w];
-        if (q_loads > 0) {
-          ok = wait_bounded(c, bar_addr(c, BAR_Q_EMPTY), qe_par, SITE_PRODUCER);
-          qe_par ^= 1u;
-          if (!ok) break;
-        }
-        mbar_arrive_expect_tx(bar_addr(c, BAR_Q_FULL), kQBytes);
-        for (int x = 0; x < 2; ++x) {
-          // a tile that starts past the last token only holds rows that are never stored:
-          // start it at the last token so that no box lies wholly outside the tensor
-          const int32_t t0 = min(it.q0 + 32 * x, p.total_tokens - 1);
-          for (int hf = 0; hf < 2; ++hf)
-            tma_load_3d(sQ + x * kTileBytes + hf * kHalfBytes, &tmap_q, bar_addr(c, BAR_Q_FULL),
-                        64 * hf, 4 * it.g, t0);
-        }
-        ++q_loads;
-        for (int j = 0; ok && j < it.n_total; ++j) {
-          for (int kv = 0; kv < 2; ++kv) {  // K_j then V_j
-            const uint32_t slot = pos % kStages;
-            const uint32_t round = pos / kStages;
-            ok = wait_bounded(c, bar_addr(c, BAR_KV_EMPTY + slot), (round & 1u) ^ 1u,
-                              SITE_PRODUCER);
+  // Registers: launched at 168 per thread (384 x 168 = 64512). The producer/MMA warpgroup
+  // hands registers to the two softmax warpgroups: 128 x 120 + 256 x 192 = 64512, the
+  // split at which neither side spills. Only that warpgroup releases and only the softmax
+  // warpgroups take, exactly the same amount, so no increase can wait on a warp that is
+  // itself waiting; no budget is ever restored (a warp that took back registers early
+  // could starve a softmax warp's increase for good). Each role ends in its own branch
+  // at a named barrier over all threads, so no code runs under two budgets, and the waits
+  // are inlined (a called function cannot serve regions with different budgets).
+  if (warp < 4) {
+    regs_decrease<120>();
+    if (warp == 0) {
+      // ------------------------------------------------------------------ TMA producer
+      if (lane == 0) {
+        tma_prefetch_desc(&tmap_q);
+        tma_prefetch_desc(&tmap_k);
+        tma_prefetch_desc(&tmap_v);
+        uint32_t pos = 0, qe_par = 0, q_loads = 0;
+        uint32_t loaded = 0, last_par = 0;  // per slot: ever loaded, parity of its last load
+        bool ok = true;
+        for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
+          const WorkItem it = p.items[w];
+          if (q_loads > 0) {
+            ok = wait_bounded(c, bar_addr(c, BAR_Q_EMPTY), qe_par, SITE_PRODUCER);
+            qe_par ^= 1u;
             if (!ok) break;
-            const uint32_t full = bar_addr(c, BAR_KV_FULL + slot);
-            mbar_arrive_expect_tx(full, kTileBytes);
-            const CUtensorMap* map = kv == 0 ? &tmap_k : &tmap_v;
+          }
+          mbar_arrive_expect_tx(bar_addr(c, BAR_Q_FULL), kQBytes);
+          for (int x = 0; x < 2; ++x) {
+            // a tile that starts past the last token only holds rows that are never stored:
+            // start it at the last token so that no box lies wholly outside the tensor
+            const int32_t t0 = min(it.q0 + 32 * x, p.total_tokens - 1);
             for (int hf = 0; hf < 2; ++hf)
-              tma_load_3d(sRing + slot * kTileBytes + hf * kHalfBytes, map, full, 64 * hf, it.g,
-                          it.kv0 + 128 * j);
-            last_round[slot] = static_cast<int32_t>(round);
-            ++pos;
+              tma_load_3d(sQ + x * kTileBytes + hf * kHalfBytes, &tmap_q, bar_addr(c, BAR_Q_FULL),
+                          64 * hf, 4 * it.g, t0);
+          }
+          ++q_loads;
+          for (int j = 0; ok && j < it.n_total; ++j) {
+            for (int kv = 0; kv < 2; ++kv) {  // K_j then V_j
+              const uint32_t slot = pos % kStages;
+              const uint32_t round = pos / kStages;
+              ok = wait_bounded(c, bar_addr(c, BAR_KV_EMPTY + slot), (round & 1u) ^ 1u,
+                                SITE_PRODUCER);
+              if (!ok) break;
+              const uint32_t full = bar_addr(c, BAR_KV_FULL + slot);
+              mbar_arrive_expect_tx(full, kTileBytes);
+              const CUtensorMap* map = kv == 0 ? &tmap_k : &tmap_v;
+              for (int hf = 0; hf < 2; ++hf)
+                tma_load_3d(sRing + slot * kTileBytes + hf * kHalfBytes, map, full, 64 * hf, it.g,
+                            it.kv0 + 128 * j);
+              loaded |= 1u << slot;
+              last_par = (last_par & ~(1u << slot)) | ((round & 1u) << slot);
+              ++pos;
+            }
           }
         }
+        // drain: every load this thread issued must land before the CTA exits (on the normal
+        // path they all have, and these waits return at once)
+        for (int s = 0; s < kStages; ++s)
+          if (loaded & (1u << s)) wait_drain(c, bar_addr(c, BAR_KV_FULL + s), (last_par >> s) & 1u);
+        if (q_loads > 0) wait_drain(c, bar_addr(c, BAR_Q_FULL), (q_loads - 1) & 1u);
       }
-      // drain: every load this thread issued must land before the CTA exits (on the normal
-      // path they all have, and these waits return at once)
-      for (int s = 0; s < kStages; ++s)
-        if (last_round[s] >= 0)
-          wait_drain(c, bar_addr(c, BAR_KV_FULL + s), static_cast<uint32_t>(last_round[s]) & 1u);
-      if (q_loads > 0) wait_drain(c, bar_addr(c, BAR_Q_FULL), (q_loads - 1) & 1u);
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      uint32_t pos = 0, qf_par = 0;
-      uint32_t p_par[2] = {0, 0}, oe_par[2] = {0, 0};
-      bool first = true, ok = true;
-      auto wait_kv = [&](uint32_t ps) {
-        return wait_bounded(c, bar_addr(c, BAR_KV_FULL + ps % kStages), (ps / kStages) & 1u,
-                            SITE_MMA);
-      };
-      auto slot_addr = [&](uint32_t ps) { return sRing + (ps % kStages) * kTileBytes; };
-      auto release = [&](uint32_t ps) { mma_commit(bar_addr(c, BAR_KV_EMPTY + ps % kStages)); };
-      // wait until softmax X has written P (and rescaled O); before the first PV of an item
-      // also wait until the previous item's epilogue has read O
-      auto wait_p = [&](int x, bool first_pv) {
-        if (!wait_bounded(c, bar_addr(c, BAR_P_FULL + x), p_par[x], SITE_MMA)) return false;
-        p_par[x] ^= 1u;
-        if (first_pv && !first) {
-          if (!wait_bounded(c, bar_addr(c, BAR_O_EMPTY + x), oe_par[x], SITE_MMA)) return false;
-          oe_par[x] ^= 1u;
-        }
-        tc_fence_after();
-        return true;
-      };
-      for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
-        const WorkItem it = p.items[w];
-        const int n = it.n_total;
-        if (!(ok = wait_bounded(c, bar_addr(c, BAR_Q_FULL), qf_par, SITE_MMA))) break;
-        qf_par ^= 1u;
-        uint32_t kpos = pos++;
-        if (!(ok = wait_kv(kpos))) break;
-        tc_fence_after();
-        issue_qk(tmem + col_s(0), sQ, slot_addr(kpos));
-        mma_commit(bar_addr(c, BAR_S_FULL + 0));
-        issue_qk(tmem + col_s(1), sQ + kTileBytes, slot_addr(kpos));
-        mma_commit(bar_addr(c, BAR_S_FULL + 1));
-        if (n == 1) mma_commit(bar_addr(c, BAR_Q_EMPTY));
-        release(kpos);
-        for (int j = 1; j < n; ++j) {
-          const uint32_t vpos = pos++;
-          kpos = pos++;
-          if (!(ok = wait_kv(vpos) && wait_kv(kpos))) break;
-          if (!(ok = wait_p(0, j == 1))) break;
-          issue_pv(tmem + col_o(0), tmem + col_s(0), slot_addr(vpos), j > 1);
+      __syncwarp();
+    } else if (warp == 1) {
+      // ------------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        uint32_t pos = 0, qf_par = 0;
+        uint32_t p_par[2] = {0, 0}, oe_par[2] = {0, 0};
+        bool first = true, ok = true;
+        auto wait_kv = [&](uint32_t ps) {
+          return wait_bounded(c, bar_addr(c, BAR_KV_FULL + ps % kStages), (ps / kStages) & 1u,
+                              SITE_MMA);
+        };
+        auto slot_addr = [&](uint32_t ps) { return sRing + (ps % kStages) * kTileBytes; };
+        auto release = [&](uint32_t ps) { mma_commit(bar_addr(c, BAR_KV_EMPTY + ps % kStages)); };
+        // wait until softmax X has written P (and rescaled O); before the first PV of an item
+        // also wait until the previous item's epilogue has read O
+        auto wait_p = [&](int x, bool first_pv) {
+          if (!wait_bounded(c, bar_addr(c, BAR_P_FULL + x), p_par[x], SITE_MMA)) return false;
+          p_par[x] ^= 1u;
+          if (first_pv && !first) {
+            if (!wait_bounded(c, bar_addr(c, BAR_O_EMPTY + x), oe_par[x], SITE_MMA)) return false;
+            oe_par[x] ^= 1u;
+          }
+          tc_fence_after();
+          return true;
+        };
+        for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
+          const WorkItem it = p.items[w];
+          const int n = it.n_total;
+          if (!(ok = wait_bounded(c, bar_addr(c, BAR_Q_FULL), qf_par, SITE_MMA))) break;
+          qf_par ^= 1u;
+          uint32_t kpos = pos++;
+          if (!(ok = wait_kv(kpos))) break;
+          tc_fence_after();
           issue_qk(tmem + col_s(0), sQ, slot_addr(kpos));
           mma_commit(bar_addr(c, BAR_S_FULL + 0));
-          if (!(ok = wait_p(1, j == 1))) break;
-          issue_pv(tmem + col_o(1), tmem + col_s(1), slot_addr(vpos), j > 1);
-          release(vpos);
           issue_qk(tmem + col_s(1), sQ + kTileBytes, slot_addr(kpos));
           mma_commit(bar_addr(c, BAR_S_FULL + 1));
-          if (j == n - 1) mma_commit(bar_addr(c, BAR_Q_EMPTY));
+          if (n == 1) mma_commit(bar_addr(c, BAR_Q_EMPTY));
           release(kpos);
+          for (int j = 1; j < n; ++j) {
+            const uint32_t vpos = pos++;
+            kpos = pos++;
+            if (!(ok = wait_kv(vpos) && wait_kv(kpos))) break;
+            if (!(ok = wait_p(0, j == 1))) break;
+            issue_pv(tmem + col_o(0), tmem + col_s(0), slot_addr(vpos), j > 1);
+            issue_qk(tmem + col_s(0), sQ, slot_addr(kpos));
+            mma_commit(bar_addr(c, BAR_S_FULL + 0));
+            if (!(ok = wait_p(1, j == 1))) break;
+            issue_pv(tmem + col_o(1), tmem + col_s(1), slot_addr(vpos), j > 1);
+            release(vpos);
+            issue_qk(tmem + col_s(1), sQ + kTileBytes, slot_addr(kpos));
+            mma_commit(bar_addr(c, BAR_S_FULL + 1));
+            if (j == n - 1) mma_commit(bar_addr(c, BAR_Q_EMPTY));
+            release(kpos);
+          }
+          if (!ok) break;
+          const uint32_t vpos = pos++;
+          if (!(ok = wait_kv(vpos))) break;
+          if (!(ok = wait_p(0, n == 1))) break;
+          issue_pv(tmem + col_o(0), tmem + col_s(0), slot_addr(vpos), n > 1);
+          mma_commit(bar_addr(c, BAR_O_FULL + 0));
+          if (!(ok = wait_p(1, n == 1))) break;
+          issue_pv(tmem + col_o(1), tmem + col_s(1), slot_addr(vpos), n > 1);
+          mma_commit(bar_addr(c, BAR_O_FULL + 1));
+          release(vpos);
+          first = false;
         }
-        if (!ok) break;
-        const uint32_t vpos = pos++;
-        if (!(ok = wait_kv(vpos))) break;
-        if (!(ok = wait_p(0, n == 1))) break;
-        issue_pv(tmem + col_o(0), tmem + col_s(0), slot_addr(vpos), n > 1);
-        mma_commit(bar_addr(c, BAR_O_FULL + 0));
-        if (!(ok = wait_p(1, n == 1))) break;
-        issue_pv(tmem + col_o(1), tmem + col_s(1), slot_addr(vpos), n > 1);
-        mma_commit(bar_addr(c, BAR_O_FULL + 1));
-        release(vpos);
-        first = false;
+        // every MMA this thread issued must complete before tensor memory is freed
+        mma_commit(bar_addr(c, BAR_DRAIN));
+        wait_drain(c, bar_addr(c, BAR_DRAIN), 0);
       }
-      // every MMA this thread issued must complete before tensor memory is freed
-      mma_commit(bar_addr(c, BAR_DRAIN));
-      wait_drain(c, bar_addr(c, BAR_DRAIN), 0);
+      __syncwarp();
     }
-    __syncwarp();
-  } else if (warp >= 4) {
+    // end of the producer/MMA warpgroup: wait for every role, then free tensor memory
+    tc_fence_before();
+    named_bar_sync(1, kThreads);
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc(tmem, kTmemCols);
+    }
+  } else {
+    regs_increase<192>();
     // ------------------------------------------------------------------ softmax
     const int x = (warp - 4) >> 2;      // tile
     const int quarter = warp & 3;       // tensor-memory lanes 32*quarter .. +31
@@ -362,40 +428,58 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 128; ++e)
             if (e >= nvis) s[e] = -INFINITY;
         }
-        float mx = s[0];
+        // row max: 8 independent chains of 16 scores (three-input max), then a tree; a
+        // single 128-long chain would expose its whole latency with one softmax warp per
+        // scheduler
+        float m8[8];
 #pragma unroll
-        for (int e = 1; e < 128; ++e) mx = fmaxf(mx, s[e]);
+        for (int i = 0; i < 8; ++i) {
+          const float* c16 = s + 16 * i;
+          float m = fmax3(c16[0], c16[1], c16[2]);
+#pragma unroll
+          for (int e = 3; e < 15; e += 2) m = fmax3(m, c16[e], c16[e + 1]);
+          m8[i] = fmaxf(m, c16[15]);
+        }
+        const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]),
+                               fmaxf(m8[6], m8[7]));
         const float m_new = fmaxf(m_used, mx);
+        float alpha = 1.f;
+        bool rescale = false;
         if (j == 0) {
           m_used = m_new;
         } else if (__any_sync(0xffffffffu, (m_new - m_used) * sl2 > 8.0f)) {
-          // warp-uniform: the tensor-memory loads and stores below are warp-collective, so
-          // when any row of the warp needs it, every row rescales (by its own factor <= 1)
-          const float alpha = ex2_approx((m_used - m_new) * sl2);
-          l *= alpha;
+          // warp-uniform: the tensor-memory loads and stores of the O rescale are
+          // warp-collective, so when any row of the warp needs it every row rescales (by
+          // its own factor <= 1)
+          alpha = ex2_approx((m_used - m_new) * sl2);
           m_used = m_new;
+          rescale = true;
+        }
+        const float mb = m_used * sl2;
+        float l4[4];
+        if (j < it.n_full)
+          exp_store_p<true>(s, sl2, mb, tS, l4);   // no -inf here: the polynomial may be used
+        else
+          exp_store_p<false>(s, sl2, mb, tS, l4);  // masked scores: MUFU gives exact zeros
+        l = fmaf(l, alpha, (l4[0] + l4[1]) + (l4[2] + l4[3]));
+        if (rescale) {
+          // O may be touched now: the PV of the previous block completed before S of this
+          // one (one commit tracks both), and the PV of this block waits for P_FULL below
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
             uint32_t o[32];
             tmem_ld32(tO + 32 * ch, o);
             tmem_wait_ld();
+            const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            for (int e = 0; e < 32; e += 2) {
+              float lo, hi;
+              f2_unpack(fmul2(f2_pack(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2), lo, hi);
+              o[e] = __float_as_uint(lo);
+              o[e + 1] = __float_as_uint(hi);
+            }
             tmem_st32(tO + 32 * ch, o);
           }
-        }
-        const float mb = m_used * sl2;
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {  // 32 keys -> 16 packed columns at a time
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float p0 = ex2_approx(fmaf(s[32 * q4 + 2 * e], sl2, -mb));
-            const float p1 = ex2_approx(fmaf(s[32 * q4 + 2 * e + 1], sl2, -mb));
-            l += p0 + p1;
-            pk[e] = pack_bf16x2(p0, p1);
-          }
-          tmem_st16(tS + 16 * q4, pk);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -431,13 +515,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar_addr(c, BAR_O_EMPTY + x));
     }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tc_fence_before();
+    named_bar_sync(1, kThreads);  // pairs with the producer/MMA warpgroup's barrier
   }
 }
 

@@ -1,0 +1,59 @@
+// 2^x evaluated on the FMA pipe, to take part of the softmax's exponentials off the MUFU.
+//
+// Method (Cody-Waite style range reduction, then a polynomial): x = n + f with
+// n = round(x) and f in [-0.5, 0.5]. Adding 1.5 * 2^23 to x rounds it to an integer and
+// leaves n in the low mantissa bits of the sum t, so t - 1.5 * 2^23 is n exactly and
+// f = x - n is exact. 2^f comes from a degree-3 polynomial whose coefficients are a
+// minimax fit (Remez exchange on the relative error) of 2^f on [-0.5, 0.5] made for this
+// library; its maximum relative error, float32 evaluation included, is 7.5e-5 -- far below
+// the 2^-9 rounding of the bf16 probabilities the result feeds. 2^n is applied by adding n
+// to the exponent field (the low bits of t shifted left by 23 are n << 23).
+//
+// Valid for x <= 8 (the online softmax never exponentiates above 2^8); inputs below -125
+// are clamped to -125, giving 2^-125 (about 2.4e-38) instead of a smaller value. Callers
+// that need exact zeros for -infinity use the MUFU instruction instead.
+#pragma once
+
+#include <cstdint>
+#include <cstring>
+
+#ifdef __CUDACC__
+#define HGX_HD __host__ __device__ __forceinline__
+#else
+#define HGX_HD inline
+#endif
+
+namespace hgx {
+
+HGX_HD uint32_t f2u(float x) {
+#ifdef __CUDA_ARCH__
+  return __float_as_uint(x);
+#else
+  uint32_t u;
+  std::memcpy(&u, &x, 4);
+  return u;
+#endif
+}
+
+HGX_HD float u2f(uint32_t u) {
+#ifdef __CUDA_ARCH__
+  return __uint_as_float(u);
+#else
+  float x;
+  std::memcpy(&x, &u, 4);
+  return x;
+#endif
+}
+
+HGX_HD float exp2_poly3(float x) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  x = fmaxf(x, -125.0f);
+  const float t = x + kShift;
+  const float f = x - (t - kShift);
+  float p = fmaf(0.0551716685295105f, f, 0.2426111251115799f);
+  p = fmaf(p, f, 0.6932609677314758f);
+  p = fmaf(p, f, 0.9999280571937561f);
+  return u2f(f2u(p) + (f2u(t) << 23));
+}
+
+}  // namespace hgx

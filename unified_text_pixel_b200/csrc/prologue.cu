@@ -11,8 +11,9 @@
 // contiguous bytes; lanes j and j + 8 of a half-warp hold the partners (k, k + 64) of a
 // rotation and swap values with one shuffle. Angles are computed once per (token, k) in
 // fp64 (positions reach ~10^4 rad, far outside the range where a float angle keeps
-// precision) and shared by all 40 heads through shared memory. HBM-bound: every byte of
-// q and k is read once and written once.
+// precision) and shared by all 40 heads through shared memory; they are computed while
+// the thread's loads (all issued first, 160 bytes per thread) are in flight. HBM-bound:
+// every byte of q and k is read once and written once.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -48,45 +49,59 @@ __device__ __forceinline__ uint4 pack8(const float (&y)[8]) {
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+constexpr int kUnits = kTok * kHeads / (kThreads / 16);  // (token, head) pairs per half-warp
+
 __global__ void __launch_bounds__(kThreads) prologue_kernel(
     __nv_bfloat16* __restrict__ q, __nv_bfloat16* __restrict__ k,
     const int32_t* __restrict__ pos, const __nv_bfloat16* __restrict__ wq,
     const __nv_bfloat16* __restrict__ wk, int32_t T, float eps, const RopeTables tab) {
   __shared__ float2 cs[kTok][kHalf];  // (cos, sin) per token and frequency
   const int t0 = blockIdx.x * kTok;
+  const int j = threadIdx.x & 15;  // 16-byte chunk of the head: features 8j .. 8j+7
+  const int u0 = threadIdx.x >> 4;
+
+  // 1. every load of this thread first, so that kUnits x 16 bytes are in flight at once
+  uint4 raw[kUnits];
+#pragma unroll
+  for (int n = 0; n < kUnits; ++n) {
+    const int u = u0 + n * (kThreads / 16);
+    const int tl = u / kHeads, hh = u % kHeads, t = t0 + tl;
+    raw[n] = make_uint4(0, 0, 0, 0);
+    if (t < T) {
+      const __nv_bfloat16* base = hh < 32 ? q + (static_cast<size_t>(t) * 32 + hh) * 128
+                                          : k + (static_cast<size_t>(t) * 8 + (hh - 32)) * 128;
+      raw[n] = *reinterpret_cast<const uint4*>(base + 8 * j);
+    }
+  }
+  // 2. angles while the loads are in flight: one (token, frequency) per thread, in fp64
   {
     const int tl = threadIdx.x / kHalf;
     const int f = threadIdx.x % kHalf;
     const int t = t0 + tl;
-    float c = 1.f, s = 0.f;
+    float c = 1.f, sn = 0.f;
     if (t < T) {
       const double phi = static_cast<double>(pos[3 * t + tab.axis[f]]) * tab.inv_freq[f];
       double sd, cd;
       sincos(phi, &sd, &cd);
       c = static_cast<float>(cd);
-      s = static_cast<float>(sd);
+      sn = static_cast<float>(sd);
     }
-    cs[tl][f] = make_float2(c, s);
+    cs[tl][f] = make_float2(c, sn);
   }
-  const int j = threadIdx.x & 15;  // 16-byte chunk of the head: features 8j .. 8j+7
   float wqv[8], wkv[8];
   unpack8(*reinterpret_cast<const uint4*>(wq + 8 * j), wqv);
   unpack8(*reinterpret_cast<const uint4*>(wk + 8 * j), wkv);
   __syncthreads();
 
+  // 3. normalise, rotate, store
   const bool low = j < 8;          // features < 64: first member of each pair
   const int f0 = (j & 7) * 8;      // frequency of this lane's first feature
-  for (int u = threadIdx.x >> 4; u < kTok * kHeads; u += kThreads / 16) {
-    const int tl = u / kHeads;
-    const int hh = u % kHeads;
-    const int t = t0 + tl;
-    const bool valid = t < T;
-    __nv_bfloat16* base = hh < 32 ? q + (static_cast<size_t>(t) * 32 + hh) * 128
-                                  : k + (static_cast<size_t>(t) * 8 + (hh - 32)) * 128;
+#pragma unroll
+  for (int n = 0; n < kUnits; ++n) {
+    const int u = u0 + n * (kThreads / 16);
+    const int tl = u / kHeads, hh = u % kHeads, t = t0 + tl;
     float x[8];
-    uint4 raw = make_uint4(0, 0, 0, 0);
-    if (valid) raw = *reinterpret_cast<const uint4*>(base + 8 * j);
-    unpack8(raw, x);
+    unpack8(raw[n], x);
     float ss = 0.f;
 #pragma unroll
     for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
@@ -104,7 +119,11 @@ __global__ void __launch_bounds__(kThreads) prologue_kernel(
       const float2 c = cs[tl][f0 + e];
       o[e] = low ? fmaf(y[e], c.x, -yp[e] * c.y) : fmaf(y[e], c.x, yp[e] * c.y);
     }
-    if (valid) *reinterpret_cast<uint4*>(base + 8 * j) = pack8(o);
+    if (t < T) {
+      __nv_bfloat16* base = hh < 32 ? q + (static_cast<size_t>(t) * 32 + hh) * 128
+                                    : k + (static_cast<size_t>(t) * 8 + (hh - 32)) * 128;
+      *reinterpret_cast<uint4*>(base + 8 * j) = pack8(o);
+    }
   }
 }
 

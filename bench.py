@@ -70,6 +70,23 @@ def _workload(name):
     return W.CONFIG_BY_NAME[name]
 
 
+def max_over_ranks(value, dist=None, device="cpu"):
+    """The largest value over all ranks (every rank gets it); the value itself at N = 1.
+    Device time of a multi-rank run is the slowest rank's."""
+    if dist is None:
+        return float(value)
+    import torch
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flops_per_rank_step, steps, world, max_ms):
+    """Throughput of the whole job: every rank runs its own replica of the workload."""
+    return world * flops_per_rank_step * steps / (max_ms * 1e-3) / 1e12
+
+
 def _descriptor(w):
     segs, cu_segs = W.flat_segments(w)
     return W.cu_seqlens(w), segs, cu_segs
@@ -300,12 +317,10 @@ def run_gpu(args):
     _log(f"timed {args.steps} steps: {elapsed_ms / args.steps:.3f} ms per step")
     pro_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
     att_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    elapsed_ms = max_over_ranks(elapsed_ms, dist, "cuda")
     if dist:
-        t = torch.tensor([elapsed_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
         dist.barrier()
-    value = ws * flops * args.steps / (elapsed_ms * 1e-3) / 1e12
+    value = whole_job_tflops(flops, args.steps, ws, elapsed_ms)
 
     # ---- e2e through hgx_attn_forward with host buffers
     pin = {n: host[n].pin_memory() for n in ("q", "k", "v", "wq", "wk")}
@@ -337,12 +352,8 @@ def run_gpu(args):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if dist:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = ws * flops * e2e_steps / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, "cuda")
+    e2e_value = whole_job_tflops(flops, e2e_steps, ws, e2e_ms)
     _log(f"e2e: {e2e_ms / e2e_steps:.3f} ms per step")
     if a.sync_status(stream) != H.HGX_OK:
         raise RuntimeError(a.last_error())

@@ -11,6 +11,7 @@ from .reference import (  # noqa: F401
     CAUSAL,
     FULL_SEQUENCE,
     FULL_IN_SEGMENT,
+    GEN_IMAGE,
     TILE_SKIP,
     TILE_PARTIAL,
     TILE_FULL,

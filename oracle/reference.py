@@ -40,7 +40,7 @@ from typing import Iterable, List, Sequence, Tuple
 
 import numpy as np
 
-CAUSAL, FULL_SEQUENCE, FULL_IN_SEGMENT = 0, 1, 2
+CAUSAL, FULL_SEQUENCE, FULL_IN_SEGMENT, GEN_IMAGE = 0, 1, 2, 3
 TILE_SKIP, TILE_PARTIAL, TILE_FULL = 0, 1, 2
 
 
@@ -131,6 +131,10 @@ def dense_mask(segments: Iterable[Tuple[int, int, int]], length: int) -> np.ndar
     causal row i (HiDream text/condition tokens; Hunyuan text tokens): j <= i.
     full_sequence row i (HiDream generation tokens): every j.
     full_in_segment row i (Hunyuan image tokens): j <= i, or j in the same segment as i.
+    gen_image row i (a Hunyuan Gen Image in a multi-Gen-Image training sequence): as
+      full_in_segment; in addition no row of a LATER segment may see a key of a gen_image
+      segment (the "hole" of "HunyuanImage 3.0 Technical Report", paper-graph-ui summary,
+      section 3.4, "The multi-generation training complication", Figure 4(b)).
     """
     seg_id = np.full(length, -1, dtype=np.int64)
     kind = np.full(length, -1, dtype=np.int64)
@@ -144,11 +148,13 @@ def dense_mask(segments: Iterable[Tuple[int, int, int]], length: int) -> np.ndar
     earlier_or_self = j <= i
     same_segment = seg_id[:, None] == seg_id[None, :]
     row_kind = kind[:, None]
-    return (
+    base = (
         ((row_kind == CAUSAL) & earlier_or_self)
         | (row_kind == FULL_SEQUENCE)
-        | ((row_kind == FULL_IN_SEGMENT) & (earlier_or_self | same_segment))
+        | (((row_kind == FULL_IN_SEGMENT) | (row_kind == GEN_IMAGE)) & (earlier_or_self | same_segment))
     )
+    hole = (kind[None, :] == GEN_IMAGE) & (seg_id[None, :] < seg_id[:, None])
+    return base & ~hole
 
 
 def unmasked_pairs(segments, length: int) -> int:

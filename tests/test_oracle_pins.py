@@ -20,7 +20,7 @@ D = 128
 
 
 # ------------------------------------------------------------------------------- masks
-@pytest.mark.parametrize("fixture", ["mask_hidream_edit_tiny.txt", "mask_gca_tiny.txt"])
+@pytest.mark.parametrize("fixture", ["mask_hidream_edit_tiny.txt", "mask_gca_tiny.txt", "mask_gca_multigen_tiny.txt"])
 def test_dense_mask_matches_hand_written_fixture(fixture):
     """Hand-derived masks from the HiDream and HunyuanImage rules (catches a swapped
     kind, an off-by-one on the diagonal, or a segment rule that looks backwards)."""
@@ -29,6 +29,35 @@ def test_dense_mask_matches_hand_written_fixture(fixture):
     expect = np.array([[c == "1" for c in row] for row in lines[1:]])
     L = expect.shape[0]
     np.testing.assert_array_equal(O.dense_mask(segs, L), expect)
+
+
+def test_single_gen_image_is_canonical_gca():
+    """With one Gen Image and nothing after it the training mask is the canonical
+    Generalized Causal Attention mask (section 3.4, "Why this works at inference")."""
+    segs_gen = [(0, 7, O.CAUSAL), (7, 9, O.GEN_IMAGE)]
+    segs_gca = [(0, 7, O.CAUSAL), (7, 9, O.FULL_IN_SEGMENT)]
+    np.testing.assert_array_equal(O.dense_mask(segs_gen, 16), O.dense_mask(segs_gca, 16))
+    # a Gen Image followed by text: the text rows lose exactly the image's keys
+    g = O.dense_mask([(0, 3, O.CAUSAL), (3, 4, O.GEN_IMAGE), (7, 5, O.CAUSAL)], 12)
+    c = O.dense_mask([(0, 3, O.CAUSAL), (3, 4, O.FULL_IN_SEGMENT), (7, 5, O.CAUSAL)], 12)
+    diff = c & ~g
+    assert not (g & ~c).any()
+    assert diff[7:, 3:7].all() and diff.sum() == 5 * 4
+
+
+def test_rows_after_a_gen_image_ignore_it():
+    """Perturbing K and V of a Gen Image leaves every later row bit-identical."""
+    segs = [(0, 10, O.CAUSAL), (10, 12, O.GEN_IMAGE), (22, 6, O.CAUSAL), (28, 9, O.GEN_IMAGE), (37, 4, O.CAUSAL)]
+    L = 41
+    q, k, v = _rand_qkv(L, 12)
+    mask = O.dense_mask(segs, L)
+    base = O.masked_gqa_attention(q, k, v, mask)
+    k2, v2 = k.copy(), v.copy()
+    k2[10:22] += 3.0
+    v2[10:22] -= 2.0
+    got = O.masked_gqa_attention(q, k2, v2, mask)
+    np.testing.assert_array_equal(got[22:], base[22:])
+    assert not np.array_equal(got[10:22], base[10:22])
 
 
 def test_unmasked_pairs_closed_forms():

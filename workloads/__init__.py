@@ -38,7 +38,9 @@ import torch
 CAUSAL = 0
 FULL_SEQUENCE = 1
 FULL_IN_SEGMENT = 2
-KIND_NAMES = {CAUSAL: "causal", FULL_SEQUENCE: "full_sequence", FULL_IN_SEGMENT: "full_in_segment"}
+GEN_IMAGE = 3
+KIND_NAMES = {CAUSAL: "causal", FULL_SEQUENCE: "full_sequence", FULL_IN_SEGMENT: "full_in_segment",
+              GEN_IMAGE: "gen_image"}
 
 NUM_Q_HEADS = 32
 NUM_KV_HEADS = 8

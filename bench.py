@@ -96,7 +96,7 @@ def _visible_pairs(w):
     # the product's own planner (host side of the library)
     import unified_text_pixel_b200 as H
 
-    return int(H.row_limits(*_descriptor(w)).astype(np.int64).sum())
+    return H.visible_pairs(*_descriptor(w))
 
 
 class ClockSampler:
@@ -187,7 +187,7 @@ def cpu_oracle_sample(w, budget_s=15.0, seed=0):
             if b not in lim_cache:
                 bsegs = [tuple(int(x) for x in segs[n]) for n in range(cu_segs[b], cu_segs[b + 1])]
                 m = O.dense_mask(bsegs, int(cu[b + 1] - cu[b]))
-                lim_cache[b] = m.sum(axis=1)
+                lim_cache[b] = m.sum(axis=1)  # visible keys per row
             flops += int(lim_cache[b][r - cu[b]]) * FLOP_PER_PAIR
     threads = _blas_threads()
     return flops / elapsed / 1e12, rows_done, elapsed, threads

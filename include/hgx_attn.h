@@ -49,7 +49,13 @@
  *   HGX_SEG_CAUSAL           j <= i
  *   HGX_SEG_FULL_SEQUENCE    every j < L_b
  *   HGX_SEG_FULL_IN_SEGMENT  j <= i, or j inside i's own segment
- * Under all three kinds the visible keys of a row form a prefix [0, lim(i)).
+ *   HGX_SEG_GEN_IMAGE        as FULL_IN_SEGMENT for its own rows; in addition its keys are
+ *                            hidden from every row of a LATER segment (the multi-Gen-Image
+ *                            training mask of HunyuanImage 3.0: paper-graph-ui summary,
+ *                            section 3.4, "The multi-generation training complication",
+ *                            Figure 4(b))
+ * Under the first three kinds the visible keys of a row form a prefix [0, lim(i)); a
+ * gen_image segment cuts a hole out of the prefix of every later row.
  *
  * Ownership and threading: the caller owns every tensor and the stream. The handle owns
  * the planner's device scratch (per-row key limits, the work list, a device error word)
@@ -87,7 +93,8 @@ typedef enum {
 typedef enum {
   HGX_SEG_CAUSAL = 0,
   HGX_SEG_FULL_SEQUENCE = 1,
-  HGX_SEG_FULL_IN_SEGMENT = 2
+  HGX_SEG_FULL_IN_SEGMENT = 2,
+  HGX_SEG_GEN_IMAGE = 3
 } hgx_seg_kind;
 
 typedef enum { HGX_TILE_SKIP = 0, HGX_TILE_PARTIAL = 1, HGX_TILE_FULL = 2 } hgx_tile_class;
@@ -146,8 +153,9 @@ hgx_status hgx_attn_attention(hgx_attn_handle* h, void* stream, const void* q, c
                               const int32_t* cu_segs_host);
 
 /* Host only (no GPU needed). Exclusive key limit lim(i) of every packed row, local to its
- * batch element: row i sees keys [0, lim(i)). lim_out has room for cap entries; T entries
- * are written. Errors: INVALID_ARG (descriptor, or cap < T). */
+ * batch element: row i sees keys [0, lim(i)) minus the keys of gen_image segments before
+ * its own segment. lim_out has room for cap entries; T entries are written. Errors:
+ * INVALID_ARG (descriptor, or cap < T). */
 hgx_status hgx_attn_row_limits(int32_t batch, const int32_t* cu_seqlens_host,
                                const hgx_segment* segs_host, const int32_t* cu_segs_host,
                                int32_t* lim_out, size_t cap);
@@ -162,6 +170,12 @@ hgx_status hgx_attn_classify(int32_t batch, const int32_t* cu_seqlens_host,
                              const hgx_segment* segs_host, const int32_t* cu_segs_host,
                              int32_t* bm_tokens, int32_t* bn_keys, uint8_t* classes_out,
                              size_t cap, size_t* n_written);
+
+/* Host only. Number of visible (query, key) pairs of the whole packed batch (holes
+ * excluded): the attention performs 4 * head_dim * num_q_heads FLOPs per pair. */
+hgx_status hgx_attn_visible_pairs(int32_t batch, const int32_t* cu_seqlens_host,
+                                  const hgx_segment* segs_host, const int32_t* cu_segs_host,
+                                  uint64_t* pairs);
 
 /* Synchronizes `stream`, then reads and clears the handle's device error word: returns
  * HGX_ERR_TIMEOUT if a bounded wait ran out since the last check, HGX_ERR_CUDA if the
@@ -188,8 +202,9 @@ hgx_status hgx_attn_set_debug(hgx_attn_handle* h, uint32_t flags, uint64_t wait_
  * Scratch (per-row key limits, work list, error word) lives in one fixed-size device array
  * inside the library (about 145 KB, held by every GPU that loads the library until the
  * process exits); planning uses fixed-size static host buffers. Hence the limits:
- * at most HGX_NOALLOC_MAX_TOKENS packed tokens and HGX_NOALLOC_MAX_BATCH batch elements;
- * larger requests return HGX_ERR_UNSUPPORTED before any device work.
+ * at most HGX_NOALLOC_MAX_TOKENS packed tokens and HGX_NOALLOC_MAX_BATCH batch elements,
+ * and no gen_image segments; other requests return HGX_ERR_UNSUPPORTED before any device
+ * work.
  *
  * Arguments are those of hgx_attn_forward with the config in place of a handle (validated
  * on every call), plus `synchronize`: when nonzero the call waits for the stream and returns

@@ -117,6 +117,29 @@ def test_forward_random_layouts_elementwise(hgx, seed):
     _compare(out.float().cpu().numpy(), ref, w.name)
 
 
+@pytest.mark.parametrize("seed", range(5))
+def test_forward_gen_image_holes_elementwise(hgx, seed):
+    """Multi-Gen-Image training layouts (HunyuanImage 3.0, section 3.4): Gen Images are
+    hidden from later rows, so key blocks of a row's prefix may be skipped or masked by a
+    hole; element by element against the oracle's dense mask."""
+    w = W.random_workload(2000 + seed, max_batch=3, max_len=1100, kinds=(0, 2, 3, 3))
+    t, _ = _device_inputs(w)
+    out, _ = _run(hgx, w)
+    ref, _, _ = _oracle_full(w, t)
+    _compare(out.float().cpu().numpy(), ref, w.name)
+
+
+def test_forward_multigen_full_size_sampled_rows(hgx):
+    w = W.CONFIG_BY_NAME["hunyuan_multigen_9088"]
+    t, _ = _device_inputs(w)
+    out, _ = _run(hgx, w)
+    rows = _sample_rows(w, seed=9)
+    segs, cu_segs = W.flat_segments(w)
+    ref = O.attention_rows(t["q"], t["k"], t["v"], W.positions(w), t["wq"], t["wk"], W.cu_seqlens(w), segs,
+                           cu_segs, rows)
+    _compare(out[rows].float().cpu().numpy(), ref, w.name)
+
+
 def test_attention_alone_on_kernel_rotated_inputs(hgx):
     """The attention kernel against the oracle's masked softmax applied to the very bf16
     q'/k' the prologue kernel wrote (isolates attention error from prologue rounding)."""

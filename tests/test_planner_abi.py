@@ -36,22 +36,27 @@ def _check_against_mask(w):
     cu, segs, cu_segs = _desc(w)
     lim = B.row_limits(cu, segs, cu_segs)
     bm, bn, classes = B.classify(cu, segs, cu_segs)
-    at = 0
+    at, pairs = 0, 0
     for b in range(len(cu) - 1):
         t0, t1 = int(cu[b]), int(cu[b + 1])
         L = t1 - t0
         bsegs = [tuple(int(x) for x in segs[n]) for n in range(cu_segs[b], cu_segs[b + 1])]
         mask = O.dense_mask(bsegs, L)
-        # every row's visible set is exactly the prefix [0, lim)
-        expect = np.zeros_like(mask)
+        pairs += int(mask.sum())
+        # every row's visible set lies in [0, lim) and reaches lim - 1 (its own segment or
+        # itself is always visible); without gen_image segments it is the whole prefix
+        has_gen = any(k == O.GEN_IMAGE for _, _, k in bsegs)
         for i in range(L):
-            expect[i, : lim[t0 + i]] = True
-        np.testing.assert_array_equal(mask, expect)
+            vis = np.nonzero(mask[i])[0]
+            assert vis.max() == lim[t0 + i] - 1
+            if not has_gen:
+                assert vis.size == lim[t0 + i]
         ref = O.tile_classes(mask, bm, bn)
         got = classes[at : at + ref.size].reshape(ref.shape)
         at += ref.size
         np.testing.assert_array_equal(got, ref)
     assert at == classes.size
+    assert B.visible_pairs(cu, segs, cu_segs) == pairs
 
 
 @pytest.mark.parametrize("cfg", range(5))
@@ -62,6 +67,17 @@ def test_limits_and_tile_classes_match_dense_mask(cfg):
 @pytest.mark.parametrize("seed", range(40))
 def test_limits_and_tile_classes_random_layouts(seed):
     _check_against_mask(W.random_workload(seed, allow_empty=(seed % 5 == 0)))
+
+
+@pytest.mark.parametrize("seed", range(30))
+def test_tile_classes_with_gen_image_holes(seed):
+    """Multi-Gen-Image training layouts: holes make FULL, PARTIAL and SKIP blocks
+    interleave; classes must still match the dense mask bit for bit."""
+    _check_against_mask(W.random_workload(1000 + seed, max_len=1400, kinds=(0, 2, 3, 3)))
+
+
+def test_multigen_workload_against_dense_mask():
+    _check_against_mask(W.CONFIG_BY_NAME["hunyuan_multigen_9088"])
 
 
 def test_tile_size_is_the_kernels():
@@ -85,7 +101,7 @@ def _status_row_limits(cu, segs, cu_segs):
 
 
 BAD = {
-    "bad_kind": ([0, 5], [[0, 5, 3]], [0, 1]),
+    "bad_kind": ([0, 5], [[0, 5, 4]], [0, 1]),
     "negative_kind": ([0, 5], [[0, 5, -1]], [0, 1]),
     "gap": ([0, 5], [[0, 2, 0], [3, 2, 1]], [0, 2]),
     "overlap": ([0, 5], [[0, 3, 0], [2, 3, 1]], [0, 2]),

@@ -14,6 +14,7 @@ from .binding import (  # noqa: F401
     HGX_SEG_CAUSAL,
     HGX_SEG_FULL_SEQUENCE,
     HGX_SEG_FULL_IN_SEGMENT,
+    HGX_SEG_GEN_IMAGE,
     HGX_TILE_SKIP,
     HGX_TILE_PARTIAL,
     HGX_TILE_FULL,
@@ -25,5 +26,6 @@ from .binding import (  # noqa: F401
     lib,
     library_path,
     row_limits,
+    visible_pairs,
     classify,
 )

@@ -13,7 +13,7 @@ from typing import Optional, Sequence, Tuple
 import numpy as np
 
 HGX_OK, HGX_ERR_INVALID_ARG, HGX_ERR_UNSUPPORTED, HGX_ERR_OOM, HGX_ERR_CUDA, HGX_ERR_TIMEOUT = range(6)
-HGX_SEG_CAUSAL, HGX_SEG_FULL_SEQUENCE, HGX_SEG_FULL_IN_SEGMENT = 0, 1, 2
+HGX_SEG_CAUSAL, HGX_SEG_FULL_SEQUENCE, HGX_SEG_FULL_IN_SEGMENT, HGX_SEG_GEN_IMAGE = 0, 1, 2, 3
 HGX_TILE_SKIP, HGX_TILE_PARTIAL, HGX_TILE_FULL = 0, 1, 2
 HGX_DEBUG_CHECKED, HGX_DEBUG_STALL_TEST = 1, 2
 
@@ -53,6 +53,7 @@ _SIGS = {
     "hgx_attn_attention": (ctypes.c_int, [ctypes.c_void_p] * 6 + [ctypes.c_int32] + [ctypes.c_void_p] * 3),
     "hgx_attn_row_limits": (ctypes.c_int, [ctypes.c_int32] + [ctypes.c_void_p] * 4 + [ctypes.c_size_t]),
     "hgx_attn_classify": (ctypes.c_int, [ctypes.c_int32] + [ctypes.c_void_p] * 6 + [ctypes.c_size_t, ctypes.c_void_p]),
+    "hgx_attn_visible_pairs": (ctypes.c_int, [ctypes.c_int32] + [ctypes.c_void_p] * 4),
     "hgx_attn_sync_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     "hgx_attn_set_debug": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_uint32, ctypes.c_uint64]),
 }
@@ -98,6 +99,16 @@ def row_limits(cu_seqlens, segs, cu_segs) -> np.ndarray:
     if st != HGX_OK:
         raise HgxError(st, "hgx_attn_row_limits")
     return out
+
+
+def visible_pairs(cu_seqlens, segs, cu_segs) -> int:
+    """Visible (query, key) pairs of the packed batch, Gen Image holes excluded."""
+    cu, sg, cs = _descriptor(cu_seqlens, segs, cu_segs)
+    out = ctypes.c_uint64()
+    st = lib().hgx_attn_visible_pairs(len(cu) - 1, _ptr(cu), _ptr(sg), _ptr(cs), ctypes.byref(out))
+    if st != HGX_OK:
+        raise HgxError(st, "hgx_attn_visible_pairs")
+    return int(out.value)
 
 
 def classify(cu_seqlens, segs, cu_segs) -> Tuple[int, int, np.ndarray]:

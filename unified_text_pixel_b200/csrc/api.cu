@@ -40,6 +40,13 @@ struct hgx_attn_handle {
   size_t lim_cap = 0;
   hgx::WorkItem* d_items = nullptr;
   size_t items_cap = 0;
+  // Gen Image hole tables (allocated only for descriptors with gen_image segments)
+  uint32_t* d_kblocks = nullptr;
+  size_t kblocks_cap = 0;
+  int32_t* d_hole_base = nullptr;
+  size_t hole_base_cap = 0;
+  uint32_t* d_hole_masks = nullptr;
+  size_t hole_masks_cap = 0;
   uint32_t* d_err = nullptr;
   // pinned staging for the plan upload, reused once the previous upload has completed
   uint8_t* h_stage = nullptr;
@@ -147,28 +154,37 @@ hgx_status prepare_plan(hgx_attn_handle* h, cudaStream_t stream, int32_t batch,
     h->plan_device = -1;
   }
   if (h->plan_device == h->device) return HGX_OK;
-  const size_t T = static_cast<size_t>(h->plan.total_tokens);
-  const size_t n_items = h->plan.items.size();
+  const hgx::Plan& pl = h->plan;
+  // (device buffer, its capacity, host data, bytes) of every array the kernel reads
+  struct Upload {
+    void** dst;
+    size_t* cap;
+    const void* src;
+    size_t bytes;
+  } up[] = {
+      {reinterpret_cast<void**>(&h->d_lim), &h->lim_cap, pl.lim.data(), pl.lim.size() * sizeof(int32_t)},
+      {reinterpret_cast<void**>(&h->d_items), &h->items_cap, pl.items.data(),
+       pl.items.size() * sizeof(hgx::WorkItem)},
+      {reinterpret_cast<void**>(&h->d_kblocks), &h->kblocks_cap, pl.kblocks.data(),
+       pl.kblocks.size() * sizeof(uint32_t)},
+      {reinterpret_cast<void**>(&h->d_hole_base), &h->hole_base_cap, pl.hole_base.data(),
+       pl.hole_base.size() * sizeof(int32_t)},
+      {reinterpret_cast<void**>(&h->d_hole_masks), &h->hole_masks_cap, pl.hole_masks.data(),
+       pl.hole_masks.size() * sizeof(uint32_t)},
+  };
+  size_t need = 0;
+  for (const Upload& u : up) {
+    if (u.bytes > *u.cap) {
+      if (*u.dst) cudaFree(*u.dst);
+      *u.dst = nullptr;
+      *u.cap = 0;
+      if (cudaMalloc(u.dst, u.bytes) != cudaSuccess)
+        return fail(h, HGX_ERR_OOM, "cudaMalloc of the planner scratch failed");
+      *u.cap = u.bytes;
+    }
+    need += (u.bytes + 255) & ~size_t(255);
+  }
   cudaError_t e;
-  if (T > h->lim_cap) {
-    if (h->d_lim) cudaFree(h->d_lim);
-    h->d_lim = nullptr;
-    h->lim_cap = 0;
-    if (cudaMalloc(&h->d_lim, T * sizeof(int32_t)) != cudaSuccess)
-      return fail(h, HGX_ERR_OOM, "cudaMalloc of the row limits failed");
-    h->lim_cap = T;
-  }
-  if (n_items > h->items_cap) {
-    if (h->d_items) cudaFree(h->d_items);
-    h->d_items = nullptr;
-    h->items_cap = 0;
-    if (cudaMalloc(&h->d_items, n_items * sizeof(hgx::WorkItem)) != cudaSuccess)
-      return fail(h, HGX_ERR_OOM, "cudaMalloc of the work list failed");
-    h->items_cap = n_items;
-  }
-  const size_t lim_bytes = T * sizeof(int32_t);
-  const size_t item_off = (lim_bytes + 255) & ~size_t(255);
-  const size_t need = item_off + n_items * sizeof(hgx::WorkItem);
   // the previous upload may still be reading the staging buffer
   e = cudaEventSynchronize(h->stage_done);
   if (e != cudaSuccess) return cuda_fail(h, e, "cudaEventSynchronize");
@@ -180,16 +196,13 @@ hgx_status prepare_plan(hgx_attn_handle* h, cudaStream_t stream, int32_t batch,
       return fail(h, HGX_ERR_OOM, "cudaMallocHost of the plan staging buffer failed");
     h->stage_cap = need;
   }
-  std::memcpy(h->h_stage, h->plan.lim.data(), lim_bytes);
-  std::memcpy(h->h_stage + item_off, h->plan.items.data(), n_items * sizeof(hgx::WorkItem));
-  if (lim_bytes) {
-    e = cudaMemcpyAsync(h->d_lim, h->h_stage, lim_bytes, cudaMemcpyHostToDevice, stream);
-    if (e != cudaSuccess) return cuda_fail(h, e, "cudaMemcpyAsync (row limits)");
-  }
-  if (n_items) {
-    e = cudaMemcpyAsync(h->d_items, h->h_stage + item_off, n_items * sizeof(hgx::WorkItem),
-                        cudaMemcpyHostToDevice, stream);
-    if (e != cudaSuccess) return cuda_fail(h, e, "cudaMemcpyAsync (work list)");
+  size_t off = 0;
+  for (const Upload& u : up) {
+    if (!u.bytes) continue;
+    std::memcpy(h->h_stage + off, u.src, u.bytes);
+    e = cudaMemcpyAsync(*u.dst, h->h_stage + off, u.bytes, cudaMemcpyHostToDevice, stream);
+    if (e != cudaSuccess) return cuda_fail(h, e, "cudaMemcpyAsync (plan)");
+    off += (u.bytes + 255) & ~size_t(255);
   }
   e = cudaEventRecord(h->stage_done, stream);
   if (e != cudaSuccess) return cuda_fail(h, e, "cudaEventRecord");
@@ -227,6 +240,9 @@ hgx_status run_attention(hgx_attn_handle* h, cudaStream_t stream, const void* q,
   p.n_items = static_cast<int32_t>(h->plan.items.size());
   p.total_tokens = T;
   p.lim = h->d_lim;
+  p.kblocks = h->plan.has_holes ? h->d_kblocks : nullptr;
+  p.hole_base = h->plan.has_holes ? h->d_hole_base : nullptr;
+  p.hole_masks = h->plan.has_holes ? h->d_hole_masks : nullptr;
   p.out = out;
   p.scale_log2 = h->scale * 1.4426950408889634f;
   p.flags = h->flags;
@@ -297,6 +313,9 @@ void hgx_attn_destroy(hgx_attn_handle* h) {
   if (!h) return;
   if (h->d_lim) cudaFree(h->d_lim);
   if (h->d_items) cudaFree(h->d_items);
+  if (h->d_kblocks) cudaFree(h->d_kblocks);
+  if (h->d_hole_base) cudaFree(h->d_hole_base);
+  if (h->d_hole_masks) cudaFree(h->d_hole_masks);
   if (h->d_err) cudaFree(h->d_err);
   if (h->h_stage) cudaFreeHost(h->h_stage);
   if (h->stage_done) cudaEventDestroy(h->stage_done);
@@ -399,32 +418,25 @@ hgx_status hgx_attn_classify(int32_t batch, const int32_t* cu_seqlens_host,
   std::string err;
   hgx_status st = hgx::build_plan(batch, cu_seqlens_host, segs_host, cu_segs_host, 1, &plan, &err);
   if (st != HGX_OK) return st;
-  // one item per query block (a single KV head was requested); recover the block order
-  size_t total = 0;
-  for (int32_t b = 0; b < batch; ++b) {
-    const int64_t L = cu_seqlens_host[b + 1] - cu_seqlens_host[b];
-    total += static_cast<size_t>(((L + hgx::kBlockTokens - 1) / hgx::kBlockTokens) *
-                                 ((L + hgx::kBlockKeys - 1) / hgx::kBlockKeys));
-  }
-  if (n_written) *n_written = total;
+  std::vector<uint8_t> classes;
+  hgx::tile_classes(plan, batch, cu_seqlens_host, &classes);
+  if (n_written) *n_written = classes.size();
   if (!classes_out) return HGX_OK;
-  if (cap < total) return HGX_ERR_INVALID_ARG;
-  // items are sorted by cost; index them by (first token) to emit in order
-  std::vector<const hgx::WorkItem*> by_q0(static_cast<size_t>(plan.total_tokens), nullptr);
-  for (const hgx::WorkItem& it : plan.items) by_q0[static_cast<size_t>(it.q0)] = &it;
-  size_t at = 0;
-  for (int32_t b = 0; b < batch; ++b) {
-    const int32_t base = cu_seqlens_host[b];
-    const int32_t L = cu_seqlens_host[b + 1] - base;
-    const int32_t nkb = (L + hgx::kBlockKeys - 1) / hgx::kBlockKeys;
-    for (int32_t r0 = 0; r0 < L; r0 += hgx::kBlockTokens) {
-      const hgx::WorkItem* it = by_q0[static_cast<size_t>(base + r0)];
-      for (int32_t kb = 0; kb < nkb; ++kb)
-        classes_out[at++] = kb < it->n_full    ? HGX_TILE_FULL
-                            : kb < it->n_total ? HGX_TILE_PARTIAL
-                                               : HGX_TILE_SKIP;
-    }
-  }
+  if (cap < classes.size()) return HGX_ERR_INVALID_ARG;
+  if (!classes.empty()) std::memcpy(classes_out, classes.data(), classes.size());
+  return HGX_OK;
+}
+
+hgx_status hgx_attn_visible_pairs(int32_t batch, const int32_t* cu_seqlens_host,
+                                  const hgx_segment* segs_host, const int32_t* cu_segs_host,
+                                  uint64_t* pairs) {
+  if (!pairs) return HGX_ERR_INVALID_ARG;
+  *pairs = 0;
+  hgx::Plan plan;
+  std::string err;
+  hgx_status st = hgx::build_plan(batch, cu_seqlens_host, segs_host, cu_segs_host, 1, &plan, &err);
+  if (st != HGX_OK) return st;
+  *pairs = plan.visible_pairs;
   return HGX_OK;
 }
 

@@ -43,7 +43,10 @@ namespace {
 using namespace sm100;
 
 constexpr int kThreads = 384;
-constexpr int kStages = 4;                    // K/V ring slots
+#ifndef HGX_KV_STAGES
+#define HGX_KV_STAGES 4
+#endif
+constexpr int kStages = HGX_KV_STAGES;        // K/V ring slots
 constexpr uint32_t kTileBytes = 32768;        // 128 rows x 128 bf16
 constexpr uint32_t kHalfBytes = 16384;        // 128 rows x 64 bf16 (one 128-byte swizzle span)
 constexpr uint32_t kQBytes = 2 * kTileBytes;  // both Q tiles of an item
@@ -157,11 +160,10 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint3
   }
 }
 
-#ifndef HGX_EXP_POLY_EVERY
-// One key pair in this many takes the FMA-pipe polynomial exp2 instead of the MUFU ex2;
-// 0 = never. Measured on B200 (edit step): the softmax is limited by instruction issue,
-// not by the MUFU, and every fraction tried (1/8, 1/4, 1/2) was slower than none.
-#define HGX_EXP_POLY_EVERY 0
+#ifndef HGX_EXP_POLY_MASK
+// Bit e set: key pair e of every 16 takes the FMA-pipe polynomial exp2 instead of the MUFU
+// ex2 (fully visible blocks only). 0 = never.
+#define HGX_EXP_POLY_MASK 0
 #endif
 
 // p = 2^(s * scale_log2 - mb) for the row's 128 scores, packed to bf16 pairs and stored as
@@ -182,10 +184,8 @@ __device__ __forceinline__ void exp_store_p(const float (&s)[128], float sl2, fl
       float x0, x1;
       f2_unpack(ffma2(f2_pack(s[32 * q4 + 2 * e], s[32 * q4 + 2 * e + 1]), scale2, shift2), x0, x1);
       float p0, p1;
-      if (kPoly && HGX_EXP_POLY_EVERY > 0 &&
-          (e % (HGX_EXP_POLY_EVERY > 0 ? HGX_EXP_POLY_EVERY : 1)) == HGX_EXP_POLY_EVERY - 1) {
-        p0 = exp2_poly3(x0);
-        p1 = exp2_poly3(x1);
+      if (kPoly && ((HGX_EXP_POLY_MASK >> e) & 1)) {
+        exp2_poly3_pair(x0, x1, p0, p1);
       } else {
         p0 = ex2_approx(x0);
         p1 = ex2_approx(x1);
@@ -291,9 +291,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint32_t full = bar_addr(c, BAR_KV_FULL + slot);
               mbar_arrive_expect_tx(full, kTileBytes);
               const CUtensorMap* map = kv == 0 ? &tmap_k : &tmap_v;
-              for (int hf = 0; hf < 2; ++hf)
+              const int32_t kb =
+                it.list_off < 0 ? j : static_cast<int32_t>(p.kblocks[it.list_off + j] & kListBlockMask);
+            for (int hf = 0; hf < 2; ++hf)
                 tma_load_3d(sRing + slot * kTileBytes + hf * kHalfBytes, map, full, 64 * hf, it.g,
-                            it.kv0 + 128 * j);
+                            it.kv0 + 128 * kb);
               loaded |= 1u << slot;
               last_par = (last_par & ~(1u << slot)) | ((round & 1u) << slot);
               ++pos;
@@ -406,8 +408,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int32_t head = 4 * it.g + (row & 3);
       const bool valid = tok - it.kv0 < it.len;
       const int32_t row_lim = valid ? p.lim[tok] : it.len;
+      const bool listed = it.list_off >= 0;  // item whose rows see a Gen Image hole
+      const int32_t hbase = (listed && valid) ? p.hole_base[tok] : -1;
       float m_used = -INFINITY, l = 0.f;
       for (int j = 0; j < it.n_total; ++j) {
+        // key block and its class (read before the wait, which hides the load)
+        const uint32_t entry = listed ? p.kblocks[it.list_off + j] : 0u;
+        const int32_t kb = listed ? static_cast<int32_t>(entry & kListBlockMask) : j;
+        const bool full = listed ? (entry >> kListClassShift) == HGX_TILE_FULL : j < it.n_full;
+        uint4 hm = make_uint4(0u, 0u, 0u, 0u);
+        if (!full && hbase >= 0)
+          hm = *reinterpret_cast<const uint4*>(p.hole_masks + 4 * static_cast<size_t>(hbase + kb));
         ok = __all_sync(0xffffffffu, wait_bounded(c, bar_addr(c, BAR_S_FULL + x), s_par,
                                                    SITE_SOFTMAX));
         if (!ok) break;
@@ -422,11 +433,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int ch = 0; ch < 4; ++ch)
 #pragma unroll
           for (int e = 0; e < 32; ++e) s[32 * ch + e] = __uint_as_float(sr[ch][e]);
-        if (j >= it.n_full) {
-          const int nvis = row_lim - 128 * j;  // keys [0, nvis) of this block are visible
+        if (!full) {
+          const int nvis = row_lim - 128 * kb;  // keys [0, nvis) of this block are in the prefix
+          if (hbase >= 0) {
+            const uint32_t hw[4] = {hm.x, hm.y, hm.z, hm.w};  // keys hidden by Gen Image holes
 #pragma unroll
-          for (int e = 0; e < 128; ++e)
-            if (e >= nvis) s[e] = -INFINITY;
+            for (int e = 0; e < 128; ++e)
+              if (e >= nvis || ((hw[e >> 5] >> (e & 31)) & 1u)) s[e] = -INFINITY;
+          } else {
+#pragma unroll
+            for (int e = 0; e < 128; ++e)
+              if (e >= nvis) s[e] = -INFINITY;
+          }
         }
         // row max: 8 independent chains of 16 scores (three-input max), then a tree; a
         // single 128-long chain would expose its whole latency with one softmax warp per
@@ -455,9 +473,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_used = m_new;
           rescale = true;
         }
-        const float mb = m_used * sl2;
+        // a row whose keys so far were all hidden (a Gen Image hole before its first visible
+        // key) still has m_used = -inf: exponentiate against 0, so its masked scores give
+        // exact zeros and its first real maximum later rescales the all-zero O by 0
+        const float mb = m_used == -INFINITY ? 0.f : m_used * sl2;
         float l4[4];
-        if (j < it.n_full)
+        if (full)
           exp_store_p<true>(s, sl2, mb, tS, l4);   // no -inf here: the polynomial may be used
         else
           exp_store_p<false>(s, sl2, mb, tS, l4);  // masked scores: MUFU gives exact zeros

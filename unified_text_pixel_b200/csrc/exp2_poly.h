@@ -56,4 +56,33 @@ HGX_HD float exp2_poly3(float x) {
   return u2f(f2u(p) + (f2u(t) << 23));
 }
 
+#ifdef __CUDACC__
+// The same evaluation for two arguments at once, with the floating-point steps as paired
+// fp32 instructions (sm_100): about 10 instructions per pair instead of 2 MUFU operations.
+__device__ __forceinline__ void exp2_poly3_pair(float x0, float x1, float& p0, float& p1) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  uint64_t x, t, r, f, p, c;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(fmaxf(x0, -125.0f)), "f"(fmaxf(x1, -125.0f)));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c) : "f"(kShift));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(t) : "l"(x), "l"(c));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c) : "f"(-kShift));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(t), "l"(c));  // round(x), exact
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c) : "f"(-1.0f));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(f) : "l"(r), "l"(c), "l"(x));  // x - round(x), exact
+  uint64_t c3, c2, c1, c0;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c3) : "f"(0.0551716685295105f));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c2) : "f"(0.2426111251115799f));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c1) : "f"(0.6932609677314758f));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c0) : "f"(0.9999280571937561f));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(c3), "l"(f), "l"(c2));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(f), "l"(c1));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(f), "l"(c0));
+  float pl, ph, tl, th;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(pl), "=f"(ph) : "l"(p));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(tl), "=f"(th) : "l"(t));
+  p0 = __uint_as_float(__float_as_uint(pl) + (__float_as_uint(tl) << 23));
+  p1 = __uint_as_float(__float_as_uint(ph) + (__float_as_uint(th) << 23));
+}
+#endif
+
 }  // namespace hgx

@@ -26,6 +26,9 @@ struct AttnParams {
   int32_t n_items;
   int32_t total_tokens;
   const int32_t* lim;      // [T] exclusive key limit per packed row, local
+  const uint32_t* kblocks;     // key-block lists of list-form items (holes only)
+  const int32_t* hole_base;    // [T] row's first hole-mask index, -1 = none (holes only)
+  const uint32_t* hole_masks;  // 4 words per (segment, key block): hidden keys (holes only)
   void* out;               // bf16 [T, 32, 128]
   float scale_log2;        // softmax scale * log2(e)
   uint32_t flags;          // HGX_DEBUG_* bits

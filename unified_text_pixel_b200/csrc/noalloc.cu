@@ -153,6 +153,7 @@ hgx_status plan(int32_t batch, const int32_t* cu, const hgx_segment* segs, const
     int32_t at = 0;
     for (int32_t s = cu_segs[b]; s < cu_segs[b + 1]; ++s) {
       const hgx_segment& sg = segs[s];
+      if (sg.kind == HGX_SEG_GEN_IMAGE) return HGX_ERR_UNSUPPORTED;  // no hole tables here
       if (sg.kind < HGX_SEG_CAUSAL || sg.kind > HGX_SEG_FULL_IN_SEGMENT || sg.len < 1 ||
           sg.start != at || sg.len > L - at)
         return HGX_ERR_INVALID_ARG;
@@ -184,6 +185,7 @@ hgx_status plan(int32_t batch, const int32_t* cu, const hgx_segment* segs, const
         it.g = g;
         it.n_full = lo / hgx::kBlockKeys;
         it.n_total = (hi + hgx::kBlockKeys - 1) / hgx::kBlockKeys;
+        it.list_off = -1;  // prefix form
       }
     }
   }

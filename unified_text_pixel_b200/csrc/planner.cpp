@@ -6,7 +6,11 @@
 // Attention (paper-graph-ui summary, section 3.4, "The core rule") -- image tokens see all
 // previous tokens and their whole segment. Under each rule the keys a row sees form a
 // prefix, so one exclusive limit per row describes the mask exactly:
-//   causal: i + 1;  full_sequence: L;  full_in_segment: end of i's segment.
+//   causal: i + 1;  full_sequence: L;  full_in_segment and gen_image: end of i's segment.
+// HunyuanImage 3.0 multi-Gen-Image training (section 3.4, "The multi-generation training
+// complication", Figure 4(b)): the keys of a gen_image segment are hidden from every row of
+// a later segment. Those "holes" lie inside the row's prefix; rows that have them get a
+// bit mask of hidden keys per key block, and their work items an explicit key-block list.
 #include "planner.h"
 
 #include <algorithm>
@@ -65,7 +69,7 @@ hgx_status validate_descriptor(int32_t batch, const int32_t* cu_seqlens,
     int32_t at = 0;
     for (int32_t s = cu_segs[b]; s < cu_segs[b + 1]; ++s) {
       const hgx_segment& sg = segs[s];
-      if (sg.kind < HGX_SEG_CAUSAL || sg.kind > HGX_SEG_FULL_IN_SEGMENT) {
+      if (sg.kind < HGX_SEG_CAUSAL || sg.kind > HGX_SEG_GEN_IMAGE) {
         *err = fmt("segment %lld has invalid kind %lld", s, sg.kind);
         return HGX_ERR_INVALID_ARG;
       }
@@ -109,7 +113,7 @@ hgx_status row_limits(int32_t batch, const int32_t* cu_seqlens, const hgx_segmen
         switch (sg.kind) {
           case HGX_SEG_CAUSAL: l = i + 1; break;
           case HGX_SEG_FULL_SEQUENCE: l = L; break;
-          default: l = sg.start + sg.len; break;  // full_in_segment
+          default: l = sg.start + sg.len; break;  // full_in_segment, gen_image
         }
         (*lim)[static_cast<size_t>(base + i)] = l;
       }
@@ -117,6 +121,15 @@ hgx_status row_limits(int32_t batch, const int32_t* cu_seqlens, const hgx_segmen
   }
   return HGX_OK;
 }
+
+namespace {
+
+int popcount4(const uint32_t* m) {
+  return __builtin_popcount(m[0]) + __builtin_popcount(m[1]) + __builtin_popcount(m[2]) +
+         __builtin_popcount(m[3]);
+}
+
+}  // namespace
 
 hgx_status build_plan(int32_t batch, const int32_t* cu_seqlens, const hgx_segment* segs,
                       const int32_t* cu_segs, int32_t num_kv_heads, Plan* plan,
@@ -126,27 +139,88 @@ hgx_status build_plan(int32_t batch, const int32_t* cu_seqlens, const hgx_segmen
   plan->batch = batch;
   plan->total_tokens = batch ? cu_seqlens[batch] : 0;
   plan->items.clear();
+  plan->kblocks.clear();
+  plan->hole_base.clear();
+  plan->hole_masks.clear();
+  plan->has_holes = false;
   plan->visible_pairs = 0;
   for (int32_t x : plan->lim) plan->visible_pairs += static_cast<uint64_t>(x);
+  for (int32_t s = 0; batch > 0 && s < cu_segs[batch]; ++s)
+    if (segs[s].kind == HGX_SEG_GEN_IMAGE) plan->has_holes = true;
+  if (plan->has_holes) plan->hole_base.assign(static_cast<size_t>(plan->total_tokens), -1);
+
+  std::vector<uint8_t> cls;  // classes of one query block, per key block
   for (int32_t b = 0; b < batch; ++b) {
     const int32_t base = cu_seqlens[b];
     const int32_t L = cu_seqlens[b + 1] - base;
+    const int32_t nkb = (L + kBlockKeys - 1) / kBlockKeys;
+    // hole masks: one 128-bit mask per key block for every segment preceded by a Gen Image
+    if (plan->has_holes) {
+      std::vector<std::pair<int32_t, int32_t>> gens;  // earlier gen_image segments
+      for (int32_t s = cu_segs[b]; s < cu_segs[b + 1]; ++s) {
+        const hgx_segment& sg = segs[s];
+        if (!gens.empty()) {
+          const int32_t mbase = static_cast<int32_t>(plan->hole_masks.size() / 4);
+          plan->hole_masks.resize(plan->hole_masks.size() + 4 * static_cast<size_t>(nkb), 0u);
+          uint32_t* m = plan->hole_masks.data() + 4 * static_cast<size_t>(mbase);
+          int64_t hidden = 0;
+          for (const auto& gsg : gens) {
+            hidden += gsg.second - gsg.first;
+            for (int32_t key = gsg.first; key < gsg.second; ++key)
+              m[4 * (key / kBlockKeys) + (key % kBlockKeys) / 32] |= 1u << (key % 32);
+          }
+          for (int32_t i = sg.start; i < sg.start + sg.len; ++i) {
+            plan->hole_base[static_cast<size_t>(base + i)] = mbase;
+            plan->visible_pairs -= static_cast<uint64_t>(hidden);
+          }
+        }
+        if (sg.kind == HGX_SEG_GEN_IMAGE) gens.emplace_back(sg.start, sg.start + sg.len);
+      }
+    }
     for (int32_t r0 = 0; r0 < L; r0 += kBlockTokens) {
       const int32_t r1 = std::min(L, r0 + kBlockTokens);
       int32_t lo = INT32_MAX, hi = 0;
+      bool holes = false;
       for (int32_t i = r0; i < r1; ++i) {
         const int32_t l = plan->lim[static_cast<size_t>(base + i)];
         lo = std::min(lo, l);
         hi = std::max(hi, l);
+        if (plan->has_holes && plan->hole_base[static_cast<size_t>(base + i)] >= 0) holes = true;
       }
-      for (int32_t g = 0; g < num_kv_heads; ++g) {
-        WorkItem it{};
-        it.q0 = base + r0;
-        it.kv0 = base;
-        it.len = L;
-        it.g = g;
+      WorkItem it{};
+      it.q0 = base + r0;
+      it.kv0 = base;
+      it.len = L;
+      it.list_off = -1;
+      if (!holes) {
         it.n_full = lo / kBlockKeys;
         it.n_total = (hi + kBlockKeys - 1) / kBlockKeys;
+      } else {
+        // classify every key block from each row's visible count
+        cls.assign(static_cast<size_t>(nkb), HGX_TILE_SKIP);
+        for (int32_t kb = 0; kb < nkb; ++kb) {
+          bool all_full = true, all_empty = true;
+          for (int32_t i = r0; i < r1; ++i) {
+            const int32_t l = plan->lim[static_cast<size_t>(base + i)];
+            int32_t vis = std::max(0, std::min(kBlockKeys, l - kb * kBlockKeys));
+            const int32_t hb = plan->hole_base[static_cast<size_t>(base + i)];
+            // hidden keys lie before the row's own segment, so inside [0, lim)
+            if (hb >= 0) vis -= popcount4(plan->hole_masks.data() + 4 * static_cast<size_t>(hb + kb));
+            all_full = all_full && vis == kBlockKeys;
+            all_empty = all_empty && vis == 0;
+          }
+          cls[static_cast<size_t>(kb)] = all_full ? HGX_TILE_FULL : all_empty ? HGX_TILE_SKIP : HGX_TILE_PARTIAL;
+        }
+        it.n_full = -1;
+        it.list_off = static_cast<int32_t>(plan->kblocks.size());
+        for (int32_t kb = 0; kb < nkb; ++kb)
+          if (cls[static_cast<size_t>(kb)] != HGX_TILE_SKIP)
+            plan->kblocks.push_back(static_cast<uint32_t>(kb) |
+                                    (static_cast<uint32_t>(cls[static_cast<size_t>(kb)]) << kListClassShift));
+        it.n_total = static_cast<int32_t>(plan->kblocks.size()) - it.list_off;
+      }
+      for (int32_t g = 0; g < num_kv_heads; ++g) {
+        it.g = g;
         plan->items.push_back(it);
       }
     }
@@ -154,6 +228,33 @@ hgx_status build_plan(int32_t batch, const int32_t* cu_seqlens, const hgx_segmen
   std::stable_sort(plan->items.begin(), plan->items.end(),
                    [](const WorkItem& a, const WorkItem& b) { return a.n_total > b.n_total; });
   return HGX_OK;
+}
+
+void tile_classes(const Plan& plan, int32_t batch, const int32_t* cu_seqlens,
+                  std::vector<uint8_t>* out) {
+  out->clear();
+  std::vector<const WorkItem*> by_q0(static_cast<size_t>(plan.total_tokens), nullptr);
+  for (const WorkItem& it : plan.items)
+    if (it.g == 0) by_q0[static_cast<size_t>(it.q0)] = &it;
+  for (int32_t b = 0; b < batch; ++b) {
+    const int32_t base = cu_seqlens[b];
+    const int32_t L = cu_seqlens[b + 1] - base;
+    const int32_t nkb = (L + kBlockKeys - 1) / kBlockKeys;
+    for (int32_t r0 = 0; r0 < L; r0 += kBlockTokens) {
+      const WorkItem* it = by_q0[static_cast<size_t>(base + r0)];
+      const size_t at = out->size();
+      out->resize(at + static_cast<size_t>(nkb), HGX_TILE_SKIP);
+      if (it->list_off < 0) {
+        for (int32_t kb = 0; kb < nkb; ++kb)
+          (*out)[at + kb] = kb < it->n_full ? HGX_TILE_FULL : kb < it->n_total ? HGX_TILE_PARTIAL : HGX_TILE_SKIP;
+      } else {
+        for (int32_t n = 0; n < it->n_total; ++n) {
+          const uint32_t e = plan.kblocks[static_cast<size_t>(it->list_off + n)];
+          (*out)[at + (e & kListBlockMask)] = static_cast<uint8_t>(e >> kListClassShift);
+        }
+      }
+    }
+  }
 }
 
 void mrope_tables(double theta, int32_t head_dim, const int32_t section[3], double* inv_freq,

@@ -23,23 +23,38 @@ constexpr int32_t kMaxTokens = (1 << 19) - 1;
 
 // One unit of attention work: one KV head g and its 4 query heads over kBlockTokens
 // consecutive query tokens of one batch element. Layout shared with the kernel.
+//
+// Prefix form (list_off < 0): the item processes key blocks 0 .. n_total-1; blocks
+// [0, n_full) are visible to every row (no mask compare), the rest need the per-row compare.
+// List form (list_off >= 0, items whose rows see a Gen Image hole): the item processes the
+// n_total key blocks listed at kblocks[list_off ...], each entry kb | class << 24 with class
+// an hgx_tile_class (FULL or PARTIAL; skipped blocks are not listed).
 struct WorkItem {
-  int32_t q0;       // packed index of the first query token
-  int32_t kv0;      // packed index of the batch element's first token
-  int32_t len;      // tokens in the batch element
-  int32_t g;        // KV head
-  int32_t n_full;   // key blocks [0, n_full) are visible to every row: no mask compare
-  int32_t n_total;  // key blocks [n_full, n_total) need the per-row compare; the rest skip
-  int32_t pad0, pad1;
+  int32_t q0;        // packed index of the first query token
+  int32_t kv0;       // packed index of the batch element's first token
+  int32_t len;       // tokens in the batch element
+  int32_t g;         // KV head
+  int32_t n_full;    // prefix form: key blocks [0, n_full) need no compare
+  int32_t n_total;   // key blocks to process
+  int32_t list_off;  // -1: prefix form; else offset into the key-block list
+  int32_t pad;
 };
 static_assert(sizeof(WorkItem) == 32, "work item layout");
+
+constexpr uint32_t kListClassShift = 24;
+constexpr uint32_t kListBlockMask = (1u << kListClassShift) - 1;
 
 struct Plan {
   int32_t batch = 0;
   int32_t total_tokens = 0;
   std::vector<int32_t> lim;        // [T] exclusive key limit per packed row, local
   std::vector<WorkItem> items;     // sorted by n_total, longest first
-  uint64_t visible_pairs = 0;      // sum of lim over all rows
+  uint64_t visible_pairs = 0;      // visible (query, key) pairs, holes excluded
+  // Gen Image holes (empty when the descriptor has no gen_image segment):
+  std::vector<uint32_t> kblocks;   // key-block lists of list-form items
+  std::vector<int32_t> hole_base;  // [T] first mask index of the row's segment, or -1
+  std::vector<uint32_t> hole_masks;  // 4 words per (segment, key block): keys hidden
+  bool has_holes = false;
 };
 
 // Checks the packed-varlen descriptor. On failure returns INVALID_ARG with *err set.
@@ -55,6 +70,11 @@ hgx_status row_limits(int32_t batch, const int32_t* cu_seqlens, const hgx_segmen
 hgx_status build_plan(int32_t batch, const int32_t* cu_seqlens, const hgx_segment* segs,
                       const int32_t* cu_segs, int32_t num_kv_heads, Plan* plan,
                       std::string* err);
+
+// Tile classes of every (query block, key block) of every batch element in order (after
+// a successful build_plan with the same descriptor).
+void tile_classes(const Plan& plan, int32_t batch, const int32_t* cu_seqlens,
+                  std::vector<uint8_t>* out);
 
 // Frequency table of the interleaved mRoPE: inv_freq[k] = theta^(-2k/D) and the axis
 // (0 t, 1 h, 2 w) that drives frequency k.

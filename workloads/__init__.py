@@ -124,7 +124,28 @@ CONFIGS: Tuple[Workload, ...] = (
     ),
 )
 
-CONFIG_BY_NAME = {w.name: w for w in CONFIGS}
+# Beyond the five: the HunyuanImage 3.0 multi-Gen-Image TRAINING mask on the same layout as
+# hunyuan_gca_9088, both images being Gen Images (each hidden from every later token).
+EXTRA: Tuple[Workload, ...] = (
+    Workload(
+        "hunyuan_multigen_9088",
+        (
+            _segments(
+                [
+                    (512, CAUSAL, None),
+                    (4096, GEN_IMAGE, (64, 64)),
+                    (256, CAUSAL, None),
+                    (4096, GEN_IMAGE, (64, 64)),
+                    (128, CAUSAL, None),
+                ]
+            ),
+        ),
+        seed=5,
+        style="hunyuan",
+    ),
+)
+
+CONFIG_BY_NAME = {w.name: w for w in CONFIGS + EXTRA}
 
 
 def config(i: int) -> Workload:
@@ -202,10 +223,10 @@ def tensors(w: Workload, device: str = "cpu"):
     return out
 
 
-def random_workload(seed: int, max_batch: int = 3, max_len: int = 700, allow_empty: bool = False) -> Workload:
-    """A seeded random segment layout (all three kinds, ragged lengths), HiDream-style
-    positions for text and Hunyuan-style for nothing: every segment with a grid gets one
-    of shape (1, len) so that positions stay integral."""
+def random_workload(seed: int, max_batch: int = 3, max_len: int = 700, allow_empty: bool = False,
+                    kinds: Sequence[int] = (CAUSAL, FULL_SEQUENCE, FULL_IN_SEGMENT)) -> Workload:
+    """A seeded random segment layout (the given kinds, ragged lengths); every non-causal
+    segment gets a (1, len) grid so that positions stay integral."""
     rng = np.random.default_rng(seed)
     batches = []
     for _ in range(int(rng.integers(1, max_batch + 1))):
@@ -213,7 +234,7 @@ def random_workload(seed: int, max_batch: int = 3, max_len: int = 700, allow_emp
         spec = []
         for _ in range(n_seg):
             length = int(rng.integers(1, max(2, max_len // max(n_seg, 1))))
-            kind = int(rng.integers(0, 3))
+            kind = int(kinds[int(rng.integers(0, len(kinds)))])
             grid = None if kind == CAUSAL else (1, length)
             spec.append((length, kind, grid))
         batches.append(_segments(spec))

@@ -15,6 +15,9 @@ from .reference import (  # noqa: F401
     TILE_SKIP,
     TILE_PARTIAL,
     TILE_FULL,
+    ROPE_MROPE_INTERLEAVED,
+    ROPE_2D_ALTERNATING,
+    ROPE_2D_HALVES,
     bf16_to_f64,
     rms_norm,
     mrope_inv_freq,

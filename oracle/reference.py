@@ -71,30 +71,49 @@ def mrope_inv_freq(theta: float, head_dim: int) -> np.ndarray:
     return np.power(float(theta), -2.0 * k / head_dim)
 
 
-def mrope_axis_of_frequency(head_dim: int, sections: Sequence[int]) -> np.ndarray:
+ROPE_MROPE_INTERLEAVED, ROPE_2D_ALTERNATING, ROPE_2D_HALVES = 0, 1, 2
+AXIS_T, AXIS_H, AXIS_W = 0, 1, 2  # position columns; in 2D layouts y = H (row), x = W (column)
+
+
+def mrope_axis_of_frequency(head_dim: int, sections: Sequence[int], layout: int = ROPE_MROPE_INTERLEAVED) -> np.ndarray:
     """Axis (0 = t, 1 = h, 2 = w) that drives each of the D/2 frequencies.
 
-    Interleaved reading of sections (s_t, s_h, s_w): the axes take turns t, h, w over the
-    frequency index while h and w still have slots (k < 3 * s_h and k < 3 * s_w); all
-    remaining frequencies belong to t.
+    ROPE_MROPE_INTERLEAVED (model card, "3-axis interleaved mRoPE [24,20,20]"): the axes take
+      turns t, h, w over the frequency index while h and w still have slots (k < 3 * s_h and
+      k < 3 * s_w); all remaining frequencies belong to t.
+    The HunyuanImage 3.0 Generalized 2D RoPE (section 3.4) for a 2D position (x, y), x the
+    column (w) and y the row (h); its two sentences disagree, so both readings exist:
+      ROPE_2D_ALTERNATING: the printed embedding [cos(x t0), cos(y t1), ...] -- frequency k is
+        driven by x when k is even and by y when k is odd;
+      ROPE_2D_HALVES: "the first half of the frequency spectrum encodes x, the second half y"
+        -- frequencies k < D/4 by x, the rest by y.
     """
     half = head_dim // 2
+    axis = np.zeros(half, dtype=np.int64)
+    if layout == ROPE_2D_ALTERNATING:
+        for k in range(half):
+            axis[k] = AXIS_W if k % 2 == 0 else AXIS_H
+        return axis
+    if layout == ROPE_2D_HALVES:
+        for k in range(half):
+            axis[k] = AXIS_W if k < half // 2 else AXIS_H
+        return axis
     s_t, s_h, s_w = (int(s) for s in sections)
     if s_t + s_h + s_w != half:
         raise ValueError("mRoPE sections must sum to head_dim / 2")
-    axis = np.zeros(half, dtype=np.int64)
     for k in range(half):
         if k % 3 == 1 and k < 3 * s_h:
-            axis[k] = 1
+            axis[k] = AXIS_H
         elif k % 3 == 2 and k < 3 * s_w:
-            axis[k] = 2
+            axis[k] = AXIS_W
     return axis
 
 
-def mrope_angles(pos: np.ndarray, theta: float, head_dim: int, sections: Sequence[int]) -> np.ndarray:
+def mrope_angles(pos: np.ndarray, theta: float, head_dim: int, sections: Sequence[int],
+                 layout: int = ROPE_MROPE_INTERLEAVED) -> np.ndarray:
     """phi[n, k] = pos[n, axis(k)] * inv_freq[k], fp64, shape [N, D/2]."""
     pos = np.asarray(pos, dtype=np.float64).reshape(-1, 3)
-    axis = mrope_axis_of_frequency(head_dim, sections)
+    axis = mrope_axis_of_frequency(head_dim, sections, layout)
     inv = mrope_inv_freq(theta, head_dim)
     return pos[:, axis] * inv[None, :]
 
@@ -111,12 +130,13 @@ def rope_rotate_half(x: np.ndarray, phi: np.ndarray) -> np.ndarray:
     return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
 
 
-def prologue(q, k, pos, wq, wk, theta: float = 5.0e6, sections=(24, 20, 20), eps: float = 1e-6):
+def prologue(q, k, pos, wq, wk, theta: float = 5.0e6, sections=(24, 20, 20), eps: float = 1e-6,
+             layout: int = ROPE_MROPE_INTERLEAVED):
     """q' = rope(rms(q) * wq), k' = rope(rms(k) * wk), fp64. q [N,Hq,D], k [N,Hkv,D]."""
     q = bf16_to_f64(q)
     k = bf16_to_f64(k)
     D = q.shape[-1]
-    phi = mrope_angles(pos, theta, D, sections)
+    phi = mrope_angles(pos, theta, D, sections, layout)
     qn = rms_norm(q, bf16_to_f64(wq), eps)
     kn = rms_norm(k, bf16_to_f64(wk), eps)
     return rope_rotate_half(qn, phi), rope_rotate_half(kn, phi)

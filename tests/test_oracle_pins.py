@@ -257,6 +257,26 @@ def test_mrope_frequency_closed_forms():
     assert abs(inv[63] - math.exp(-(126.0 / 128.0) * math.log(5e6))) < 1e-20
 
 
+@pytest.mark.parametrize("name,layout", [("alternating", O.ROPE_2D_ALTERNATING), ("halves", O.ROPE_2D_HALVES)])
+def test_2d_rope_layouts_match_the_passage(name, layout):
+    """The two readings of the Generalized 2D RoPE, written out by hand from the passage;
+    moving x only rotates exactly the x frequencies; text on the diagonal (n, n) is 1D RoPE."""
+    row = {ln.split()[0]: ln.split()[1] for ln in read_golden("rope2d_layouts.txt")}[name]
+    axis = O.mrope_axis_of_frequency(D, (24, 20, 20), layout)
+    assert "".join("x" if a == 2 else "y" if a == 1 else "t" for a in axis) == row
+    x = np.ones((1, 1, D))
+    pos = np.array([[0, 0, 9]])  # (t, h = y, w = x)
+    y = O.rope_rotate_half(x, O.mrope_angles(pos, 5e6, D, (24, 20, 20), layout))
+    moved = np.abs(y[0, 0, : D // 2] - 1.0) > 1e-15
+    assert "".join("x" if m else "y" for m in moved) == row
+    rng = np.random.default_rng(13)
+    v = rng.standard_normal((3, 2, D))
+    ps = np.array([5, 77, 4000])
+    got = O.rope_rotate_half(v, O.mrope_angles(np.stack([ps, ps, ps], 1), 5e6, D, (24, 20, 20), layout))
+    for n, p_ in enumerate(ps):
+        np.testing.assert_allclose(got[n], _rope_1d_complex(v[n], float(p_), 5e6), rtol=0, atol=1e-10)
+
+
 def test_prologue_order_norm_then_rotate():
     """RMSNorm before RoPE: the output's RMS per head equals that of rms(x) * w at every
     position (rotation keeps norms), so changing the position never changes it."""

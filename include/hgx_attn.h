@@ -28,7 +28,9 @@
  * the square root, weight multiplies, one weight vector shared by all heads; RMSNorm
  * before RoPE; query head h reads KV head h / (Hq / Hkv); "interleaved [24,20,20]" drives
  * frequency k by axis h when k % 3 == 1 and k < 60, by axis w when k % 3 == 2 and k < 60,
- * and by axis t otherwise.
+ * and by axis t otherwise. HunyuanImage 3.0's Generalized 2D RoPE (same report, section
+ * 3.4) is printed as [cos(x t0), cos(y t1), ...] but described as "first half x, second half
+ * y"; both are offered (hgx_rope_layout), with x the w column and y the h column of pos.
  *
  * Data layout (all device tensors row-major, packed varlen: the tokens of all batch
  * elements back to back, T = cu_seqlens[batch] tokens in total):
@@ -105,6 +107,12 @@ typedef struct {
   int32_t kind;  /* hgx_seg_kind */
 } hgx_segment;
 
+typedef enum {
+  HGX_ROPE_MROPE_INTERLEAVED = 0, /* 3-axis (t, h, w) interleaved over mrope_section */
+  HGX_ROPE_2D_ALTERNATING = 1,    /* 2D (x = w, y = h): frequency k by x if k even, else y */
+  HGX_ROPE_2D_HALVES = 2          /* 2D: frequencies k < head_dim / 4 by x, the rest by y */
+} hgx_rope_layout;
+
 typedef struct {
   int32_t num_q_heads;      /* must be 32 */
   int32_t num_kv_heads;     /* must be 8 */
@@ -113,6 +121,7 @@ typedef struct {
   int32_t mrope_section[3]; /* (t, h, w) frequency counts, sum head_dim / 2; {24, 20, 20} */
   float rms_eps;            /* >= 0; 1e-6 */
   float softmax_scale;      /* > 0, or 0 for 1 / sqrt(head_dim) */
+  int32_t rope_layout;      /* hgx_rope_layout; mrope_section applies to the interleaved one */
 } hgx_attn_config;
 
 typedef struct hgx_attn_handle hgx_attn_handle;
@@ -140,6 +149,20 @@ hgx_status hgx_attn_forward(hgx_attn_handle* h, void* stream, void* q, void* k, 
                             void* out, const int32_t* pos_thw, const void* q_norm_w,
                             const void* k_norm_w, int32_t batch, const int32_t* cu_seqlens_host,
                             const hgx_segment* segs_host, const int32_t* cu_segs_host);
+
+/* One denoising step with a reused prefix (the text before <|tms|> of the HiDream-O1
+ * layout is causal, so its keys, values and outputs are the same in all 100 forwards of an
+ * image: "hidream-o1-p100a" model card, "What this model is" and "Performance"). Only rows
+ * [first_rows_host[b], L_b) of element b are computed: their q and k get the prologue,
+ * their out rows are written. Rows before first_rows_host[b] keep their out, and their k
+ * must already hold k' (e.g. from an earlier call); their q is not read. Every reused row
+ * must see no key at or after first_rows_host[b] (HGX_ERR_INVALID_ARG otherwise). Other
+ * arguments as hgx_attn_forward; first_rows_host int32 [batch], host. */
+hgx_status hgx_attn_forward_from(hgx_attn_handle* h, void* stream, void* q, void* k,
+                                 const void* v, void* out, const int32_t* pos_thw,
+                                 const void* q_norm_w, const void* k_norm_w, int32_t batch,
+                                 const int32_t* cu_seqlens_host, const hgx_segment* segs_host,
+                                 const int32_t* cu_segs_host, const int32_t* first_rows_host);
 
 /* The prologue alone on total_tokens tokens (q and k overwritten with q' and k'). */
 hgx_status hgx_attn_prologue(hgx_attn_handle* h, void* stream, void* q, void* k,

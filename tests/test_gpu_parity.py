@@ -95,6 +95,23 @@ def test_prologue_matches_oracle(hgx, case):
         assert bool((pad == 7.0).all())
 
 
+@pytest.mark.parametrize("layout", [1, 2])
+def test_prologue_2d_rope_layouts(hgx, layout):
+    """HunyuanImage 3.0 Generalized 2D RoPE, both readings (x = w column, y = h column), on
+    the Hunyuan-style positions (text on the diagonal, image tokens on a 2D grid)."""
+    H, _ = hgx
+    a = H.Attention(rope_layout=layout)
+    w = W.Workload("gca_2d", (W._segments([(40, W.CAUSAL, None), (64, W.FULL_IN_SEGMENT, (8, 8)), (9, W.CAUSAL, None)]),),
+                   seed=17, style="hunyuan")
+    t, d = _device_inputs(w)
+    a.prologue(d["q"], d["k"], d["pos"], d["wq"], d["wk"])
+    assert a.sync_status() == H.HGX_OK
+    qr, kr = O.prologue(t["q"], t["k"], W.positions(w), t["wq"], t["wk"], layout=layout)
+    np.testing.assert_allclose(d["q"].float().cpu().numpy(), qr, rtol=2.0 ** -8, atol=1e-5)
+    np.testing.assert_allclose(d["k"].float().cpu().numpy(), kr, rtol=2.0 ** -8, atol=1e-5)
+    a.close()
+
+
 # ------------------------------------------------------------------------------ attention
 @pytest.mark.parametrize("cfg", [0, 1])
 def test_forward_small_configs_elementwise(hgx, cfg):
@@ -194,6 +211,43 @@ def test_online_rescale_path_with_divergent_rows(hgx):
         err = np.abs(got[t0:t1] - ref)
         assert np.isfinite(got[t0:t1]).all()
         assert err.max() <= ATOL_MAX and err.mean() <= ATOL_MEAN, (float(err.max()), float(err.mean()))
+
+
+def test_forward_from_reuses_the_text_prefix(hgx):
+    """A denoising step that keeps the text before <|tms|> (causal, so unchanged across
+    steps) and recomputes the rest: bit-identical to a full forward on the same inputs, and
+    the reused output rows are left untouched."""
+    H, a = hgx
+    w = W.config(1)  # CFG pair: (128 text + <|tms|>, 1024 patches), (16 text + <|tms|>, 1024)
+    cu, segs, cu_segs = _desc(w)
+    first = [128, 16]
+    t0 = W.tensors(w)
+    t1 = W.tensors(W.Workload(w.name, w.batches, seed=w.seed + 100, style=w.style))
+    pos = torch.from_numpy(W.positions(w)).cuda()
+    wq, wk = t0["wq"].cuda(), t0["wk"].cuda()
+    # step 0: full forward; k is rotated in place
+    q0, k0, v0 = t0["q"].cuda(), t0["k"].cuda(), t0["v"].cuda()
+    out0 = torch.empty_like(q0)
+    a.forward(q0, k0, v0, out0, pos, wq, wk, cu, segs, cu_segs)
+    suffix = torch.zeros(w.total_tokens, dtype=torch.bool)
+    for b in range(len(cu) - 1):
+        suffix[int(cu[b]) + first[b] : int(cu[b + 1])] = True
+    mix = lambda new, old: torch.where(suffix[:, None, None], new, old)  # noqa: E731
+    # step 1: new suffix inputs; the prefix keeps its rotated k and its outputs
+    q1 = mix(t1["q"], t0["q"]).cuda()
+    k1 = torch.where(suffix[:, None, None].cuda(), t1["k"].cuda(), k0)
+    v1 = mix(t1["v"], t0["v"]).cuda()
+    out1 = out0.clone()
+    a.forward_from(q1, k1, v1, out1, pos, wq, wk, cu, segs, cu_segs, first)
+    assert a.sync_status() == H.HGX_OK
+    # the same step computed from scratch
+    qr, kr, vr = mix(t1["q"], t0["q"]).cuda(), mix(t1["k"], t0["k"]).cuda(), mix(t1["v"], t0["v"]).cuda()
+    out_r = torch.empty_like(qr)
+    a.forward(qr, kr, vr, out_r, pos, wq, wk, cu, segs, cu_segs)
+    assert a.sync_status() == H.HGX_OK
+    assert torch.equal(out1, out_r)
+    assert torch.equal(out1[~suffix.cuda()], out0[~suffix.cuda()])
+    assert torch.equal(k1, kr)  # the recomputed rows were rotated like a full prologue
 
 
 def test_single_token_returns_its_value(hgx):

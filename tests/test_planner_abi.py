@@ -152,6 +152,11 @@ def test_create_rejects_bad_configs():
     assert status(mrope_section=[24, 20, 21]) == B.HGX_ERR_INVALID_ARG
     assert status(mrope_section=[4, 30, 30]) == B.HGX_ERR_UNSUPPORTED
     assert L.hgx_attn_create(None, ctypes.byref(ctypes.c_void_p())) == B.HGX_ERR_INVALID_ARG
+    assert status(rope_layout=3) == B.HGX_ERR_INVALID_ARG
+    assert status(rope_layout=-1) == B.HGX_ERR_INVALID_ARG
+    # the 2D layouts ignore mrope_section
+    assert status(rope_layout=B.HGX_ROPE_2D_ALTERNATING, mrope_section=[4, 30, 30]) == B.HGX_OK
+    assert status(rope_layout=B.HGX_ROPE_2D_HALVES, mrope_section=[0, 0, 0]) == B.HGX_OK
 
 
 def _fake(addr):
@@ -193,6 +198,26 @@ def test_forward_rejects_before_device_work():
     assert e.value.status == B.HGX_ERR_INVALID_ARG and "overlap" in str(e.value)
     # an empty batch returns OK without touching the device (works without a GPU)
     a.forward(*[None] * 7, [0, 0], np.zeros((0, 3)), [0, 0], stream=0)
+    a.close()
+
+
+def test_forward_from_checks_the_reused_prefix_before_device_work():
+    """A reused (cached) row must not see a recomputed key: on the 2048^2 edit layout the
+    257 causal text rows may be reused, any generation row may not."""
+    a = B.Attention()
+    w = W.config(3)
+    cu, segs, cu_segs = _desc(w)
+    good = [_fake(0x40000000 * (i + 1)) for i in range(7)]
+    for first, ok in ((0, True), (256, True), (257, True), (258, False), (8449, True), (-1, False), (8450, False)):
+        try:
+            a.forward_from(*good, cu, segs, cu_segs, [first], stream=0)
+            raised = None
+        except B.HgxError as e:
+            raised = e
+        if ok:  # passes the checks, then fails only because this machine has no GPU
+            assert raised is not None and raised.status == B.HGX_ERR_CUDA, (first, raised)
+        else:
+            assert raised is not None and raised.status == B.HGX_ERR_INVALID_ARG, (first, raised)
     a.close()
 
 

@@ -20,6 +20,9 @@ from .binding import (  # noqa: F401
     HGX_TILE_FULL,
     HGX_DEBUG_CHECKED,
     HGX_DEBUG_STALL_TEST,
+    HGX_ROPE_MROPE_INTERLEAVED,
+    HGX_ROPE_2D_ALTERNATING,
+    HGX_ROPE_2D_HALVES,
     HgxError,
     AttnConfig,
     Attention,

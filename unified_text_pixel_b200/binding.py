@@ -16,6 +16,7 @@ HGX_OK, HGX_ERR_INVALID_ARG, HGX_ERR_UNSUPPORTED, HGX_ERR_OOM, HGX_ERR_CUDA, HGX
 HGX_SEG_CAUSAL, HGX_SEG_FULL_SEQUENCE, HGX_SEG_FULL_IN_SEGMENT, HGX_SEG_GEN_IMAGE = 0, 1, 2, 3
 HGX_TILE_SKIP, HGX_TILE_PARTIAL, HGX_TILE_FULL = 0, 1, 2
 HGX_DEBUG_CHECKED, HGX_DEBUG_STALL_TEST = 1, 2
+HGX_ROPE_MROPE_INTERLEAVED, HGX_ROPE_2D_ALTERNATING, HGX_ROPE_2D_HALVES = 0, 1, 2
 
 _STATUS = {0: "HGX_OK", 1: "HGX_ERR_INVALID_ARG", 2: "HGX_ERR_UNSUPPORTED", 3: "HGX_ERR_OOM",
            4: "HGX_ERR_CUDA", 5: "HGX_ERR_TIMEOUT"}
@@ -38,6 +39,7 @@ class AttnConfig(ctypes.Structure):
         ("mrope_section", ctypes.c_int32 * 3),
         ("rms_eps", ctypes.c_float),
         ("softmax_scale", ctypes.c_float),
+        ("rope_layout", ctypes.c_int32),
     ]
 
 
@@ -49,6 +51,7 @@ _SIGS = {
     "hgx_attn_destroy": (None, [ctypes.c_void_p]),
     "hgx_attn_last_error": (ctypes.c_char_p, [ctypes.c_void_p]),
     "hgx_attn_forward": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_int32] + [ctypes.c_void_p] * 3),
+    "hgx_attn_forward_from": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_int32] + [ctypes.c_void_p] * 4),
     "hgx_attn_prologue": (ctypes.c_int, [ctypes.c_void_p] * 7 + [ctypes.c_int32]),
     "hgx_attn_attention": (ctypes.c_int, [ctypes.c_void_p] * 6 + [ctypes.c_int32] + [ctypes.c_void_p] * 3),
     "hgx_attn_row_limits": (ctypes.c_int, [ctypes.c_int32] + [ctypes.c_void_p] * 4 + [ctypes.c_size_t]),
@@ -146,12 +149,14 @@ def _stream_ptr(stream):
 class Attention:
     """Owns one hgx_attn_handle. Methods take torch CUDA tensors (bf16 / int32)."""
 
-    def __init__(self, config: Optional[AttnConfig] = None):
+    def __init__(self, config: Optional[AttnConfig] = None, **overrides):
         L = lib()
         cfg = AttnConfig()
         L.hgx_attn_default_config(ctypes.byref(cfg))
         if config is not None:
             cfg = config
+        for name, value in overrides.items():
+            setattr(cfg, name, value)
         self.config = cfg
         h = ctypes.c_void_p()
         st = L.hgx_attn_create(ctypes.byref(cfg), ctypes.byref(h))
@@ -188,6 +193,15 @@ class Attention:
                                     _dev_ptr(out), _dev_ptr(pos), _dev_ptr(wq), _dev_ptr(wk), len(cu) - 1,
                                     _ptr(cu), _ptr(sg), _ptr(cs))
         self._check(st, "hgx_attn_forward")
+
+    def forward_from(self, q, k, v, out, pos, wq, wk, cu_seqlens, segs, cu_segs, first_rows, stream=None):
+        """hgx_attn_forward_from: recompute rows [first_rows[b], L_b) only (reused prefix)."""
+        cu, sg, cs = _descriptor(cu_seqlens, segs, cu_segs)
+        fr = _i32(first_rows).reshape(-1)
+        st = lib().hgx_attn_forward_from(self._h, _stream_ptr(stream), _dev_ptr(q), _dev_ptr(k), _dev_ptr(v),
+                                         _dev_ptr(out), _dev_ptr(pos), _dev_ptr(wq), _dev_ptr(wk), len(cu) - 1,
+                                         _ptr(cu), _ptr(sg), _ptr(cs), _ptr(fr))
+        self._check(st, "hgx_attn_forward_from")
 
     def prologue(self, q, k, pos, wq, wk, total_tokens=None, stream=None):
         T = q.shape[0] if total_tokens is None else total_tokens

@@ -30,6 +30,7 @@ struct hgx_attn_handle {
   int32_t key_batch = -1;
   std::vector<int32_t> key_cu, key_cu_segs;
   std::vector<hgx_segment> key_segs;
+  std::vector<int32_t> key_first;  // first recomputed row per element; empty = all rows
   hgx::Plan plan;
   int plan_device = -1;
 
@@ -126,8 +127,12 @@ hgx_status ensure_device(hgx_attn_handle* h) {
 }
 
 bool same_descriptor(const hgx_attn_handle* h, int32_t batch, const int32_t* cu,
-                     const hgx_segment* segs, const int32_t* cu_segs) {
+                     const hgx_segment* segs, const int32_t* cu_segs, const int32_t* first) {
   if (h->key_batch != batch) return false;
+  if (first ? (h->key_first.size() != static_cast<size_t>(batch) ||
+               std::memcmp(h->key_first.data(), first, sizeof(int32_t) * batch) != 0)
+            : !h->key_first.empty())
+    return false;
   if (std::memcmp(h->key_cu.data(), cu, sizeof(int32_t) * (batch + 1)) != 0) return false;
   if (std::memcmp(h->key_cu_segs.data(), cu_segs, sizeof(int32_t) * (batch + 1)) != 0)
     return false;
@@ -139,18 +144,24 @@ bool same_descriptor(const hgx_attn_handle* h, int32_t batch, const int32_t* cu,
 // Builds (or reuses) the plan of this descriptor and makes sure it is on the device,
 // uploaded in stream order.
 hgx_status prepare_plan(hgx_attn_handle* h, cudaStream_t stream, int32_t batch,
-                        const int32_t* cu, const hgx_segment* segs, const int32_t* cu_segs) {
-  const bool same = same_descriptor(h, batch, cu, segs, cu_segs);
+                        const int32_t* cu, const hgx_segment* segs, const int32_t* cu_segs,
+                        const int32_t* first = nullptr) {
+  const bool same = same_descriptor(h, batch, cu, segs, cu_segs, first);
   if (!same) {
     hgx::Plan plan;
     std::string err;
-    hgx_status st = hgx::build_plan(batch, cu, segs, cu_segs, h->cfg.num_kv_heads, &plan, &err);
+    hgx_status st =
+        hgx::build_plan(batch, cu, segs, cu_segs, h->cfg.num_kv_heads, &plan, &err, first);
     if (st != HGX_OK) return fail(h, st, err);
     h->plan = std::move(plan);
     h->key_batch = batch;
     h->key_cu.assign(cu, cu + batch + 1);
     h->key_cu_segs.assign(cu_segs, cu_segs + batch + 1);
     h->key_segs.assign(segs, segs + cu_segs[batch]);
+    if (first)
+      h->key_first.assign(first, first + batch);
+    else
+      h->key_first.clear();
     h->plan_device = -1;
   }
   if (h->plan_device == h->device) return HGX_OK;
@@ -269,6 +280,7 @@ void hgx_attn_default_config(hgx_attn_config* cfg) {
   cfg->mrope_section[2] = 20;
   cfg->rms_eps = 1e-6f;
   cfg->softmax_scale = 0.f;
+  cfg->rope_layout = HGX_ROPE_MROPE_INTERLEAVED;
 }
 
 hgx_status hgx_attn_create(const hgx_attn_config* cfg, hgx_attn_handle** out) {
@@ -285,13 +297,15 @@ hgx_status hgx_attn_create(const hgx_attn_config* cfg, hgx_attn_handle** out) {
     return HGX_ERR_INVALID_ARG;
   if (cfg->num_q_heads != 32 || cfg->num_kv_heads != 8 || cfg->head_dim != 128)
     return HGX_ERR_UNSUPPORTED;
-  if (cfg->mrope_section[0] + cfg->mrope_section[1] + cfg->mrope_section[2] != cfg->head_dim / 2)
+  if (cfg->rope_layout < HGX_ROPE_MROPE_INTERLEAVED || cfg->rope_layout > HGX_ROPE_2D_HALVES)
     return HGX_ERR_INVALID_ARG;
-  {
+  if (cfg->rope_layout == HGX_ROPE_MROPE_INTERLEAVED) {
+    if (cfg->mrope_section[0] + cfg->mrope_section[1] + cfg->mrope_section[2] != cfg->head_dim / 2)
+      return HGX_ERR_INVALID_ARG;
     // the interleaved assignment must give each axis exactly its section's count
     double inv[64];
     int32_t axis[64], count[3] = {0, 0, 0};
-    hgx::mrope_tables(cfg->rope_theta, cfg->head_dim, cfg->mrope_section, inv, axis);
+    hgx::mrope_tables(cfg->rope_theta, cfg->head_dim, cfg->mrope_section, cfg->rope_layout, inv, axis);
     for (int i = 0; i < 64; ++i) ++count[axis[i]];
     for (int i = 0; i < 3; ++i)
       if (count[i] != cfg->mrope_section[i]) return HGX_ERR_UNSUPPORTED;
@@ -302,7 +316,8 @@ hgx_status hgx_attn_create(const hgx_attn_config* cfg, hgx_attn_handle** out) {
   h->scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale
                                       : static_cast<float>(1.0 / std::sqrt(double(cfg->head_dim)));
   int32_t axis[64];
-  hgx::mrope_tables(cfg->rope_theta, cfg->head_dim, cfg->mrope_section, h->rope.inv_freq, axis);
+  hgx::mrope_tables(cfg->rope_theta, cfg->head_dim, cfg->mrope_section, cfg->rope_layout,
+                    h->rope.inv_freq, axis);
   for (int i = 0; i < 64; ++i) h->rope.axis[i] = static_cast<uint8_t>(axis[i]);
   if (const char* env = std::getenv("HGX_DEBUG")) h->flags = static_cast<uint32_t>(std::atoi(env));
   *out = h;
@@ -392,6 +407,44 @@ hgx_status hgx_attn_forward(hgx_attn_handle* h, void* stream, void* q, void* k, 
       hgx::launch_prologue(s, q, k, pos_thw, q_norm_w, k_norm_w, T, h->cfg.rms_eps, h->rope);
   if (e != cudaSuccess) return cuda_fail(h, e, "prologue launch");
   if ((st = run_attention(h, s, q, k, v, out)) != HGX_OK) return st;
+  return finish(h, s);
+}
+
+hgx_status hgx_attn_forward_from(hgx_attn_handle* h, void* stream, void* q, void* k,
+                                 const void* v, void* out, const int32_t* pos_thw,
+                                 const void* q_norm_w, const void* k_norm_w, int32_t batch,
+                                 const int32_t* cu_seqlens_host, const hgx_segment* segs_host,
+                                 const int32_t* cu_segs_host, const int32_t* first_rows_host) {
+  if (!h) return HGX_ERR_INVALID_ARG;
+  h->last_error.clear();
+  std::string err;
+  int32_t T = 0;
+  hgx_status st = hgx::validate_descriptor(batch, cu_seqlens_host, segs_host, cu_segs_host,
+                                           &err, &T);
+  if (st != HGX_OK) return fail(h, st, err);
+  if ((st = hgx::check_first_rows(batch, cu_seqlens_host, segs_host, cu_segs_host, first_rows_host,
+                                  &err)) != HGX_OK)
+    return fail(h, st, err);
+  if (T == 0) return HGX_OK;
+  if ((st = check_tensors(h, {q, k, v, out, pos_thw, q_norm_w, k_norm_w})) != HGX_OK) return st;
+  const size_t qb = size_t(T) * 8192, kb = size_t(T) * 2048;
+  if (overlaps(out, qb, q, qb) || overlaps(out, qb, k, kb) || overlaps(out, qb, v, kb))
+    return fail(h, HGX_ERR_INVALID_ARG, "out overlaps q, k or v");
+  if ((st = ensure_device(h)) != HGX_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = prepare_plan(h, s, batch, cu_seqlens_host, segs_host, cu_segs_host, first_rows_host)) !=
+      HGX_OK)
+    return st;
+  for (int32_t b = 0; b < batch; ++b) {
+    const int32_t t0 = cu_seqlens_host[b] + first_rows_host[b];
+    const int32_t n = cu_seqlens_host[b + 1] - t0;
+    if (n <= 0) continue;
+    cudaError_t e = hgx::launch_prologue(
+        s, static_cast<uint8_t*>(q) + size_t(t0) * 8192, static_cast<uint8_t*>(k) + size_t(t0) * 2048,
+        pos_thw + 3 * size_t(t0), q_norm_w, k_norm_w, n, h->cfg.rms_eps, h->rope);
+    if (e != cudaSuccess) return cuda_fail(h, e, "prologue launch");
+  }
+  if (!h->plan.items.empty() && (st = run_attention(h, s, q, k, v, out)) != HGX_OK) return st;
   return finish(h, s);
 }
 

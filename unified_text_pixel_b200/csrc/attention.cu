@@ -406,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const WorkItem it = p.items[w];
       const int32_t tok = it.q0 + 32 * x + (row >> 2);
       const int32_t head = 4 * it.g + (row & 3);
-      const bool valid = tok - it.kv0 < it.len;
+      const bool valid = tok - it.kv0 < it.len && tok - it.kv0 >= it.first;
       const int32_t row_lim = valid ? p.lim[tok] : it.len;
       const bool listed = it.list_off >= 0;  // item whose rows see a Gen Image hole
       const int32_t hbase = (listed && valid) ? p.hole_base[tok] : -1;

@@ -126,7 +126,10 @@ hgx_status check_config(const hgx_attn_config* cfg) {
     return HGX_ERR_UNSUPPORTED;
   for (int i = 0; i < 3; ++i)
     if (cfg->mrope_section[i] < 0) return HGX_ERR_INVALID_ARG;
-  if (cfg->mrope_section[0] + cfg->mrope_section[1] + cfg->mrope_section[2] != 64)
+  if (cfg->rope_layout < HGX_ROPE_MROPE_INTERLEAVED || cfg->rope_layout > HGX_ROPE_2D_HALVES)
+    return HGX_ERR_INVALID_ARG;
+  if (cfg->rope_layout == HGX_ROPE_MROPE_INTERLEAVED &&
+      cfg->mrope_section[0] + cfg->mrope_section[1] + cfg->mrope_section[2] != 64)
     return HGX_ERR_INVALID_ARG;
   return HGX_OK;
 }
@@ -237,14 +240,16 @@ extern "C" hgx_status hgx_attn_forward_noalloc(const hgx_attn_config* cfg, void*
 
   hgx::RopeTables rope{};
   int32_t axis[64];
-  hgx::mrope_tables(cfg->rope_theta, cfg->head_dim, cfg->mrope_section, rope.inv_freq, axis);
+  hgx::mrope_tables(cfg->rope_theta, cfg->head_dim, cfg->mrope_section, cfg->rope_layout,
+                    rope.inv_freq, axis);
   int32_t count[3] = {0, 0, 0};
   for (int i = 0; i < 64; ++i) {
     rope.axis[i] = static_cast<uint8_t>(axis[i]);
     ++count[axis[i]];
   }
-  for (int i = 0; i < 3; ++i)
-    if (count[i] != cfg->mrope_section[i]) return HGX_ERR_UNSUPPORTED;
+  if (cfg->rope_layout == HGX_ROPE_MROPE_INTERLEAVED)
+    for (int i = 0; i < 3; ++i)
+      if (count[i] != cfg->mrope_section[i]) return HGX_ERR_UNSUPPORTED;
   if (hgx::launch_prologue(s, q, k, pos_thw, q_norm_w, k_norm_w, T, cfg->rms_eps, rope) != cudaSuccess)
     return HGX_ERR_CUDA;
 

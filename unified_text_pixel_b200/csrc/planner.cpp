@@ -122,6 +122,31 @@ hgx_status row_limits(int32_t batch, const int32_t* cu_seqlens, const hgx_segmen
   return HGX_OK;
 }
 
+hgx_status check_first_rows(int32_t batch, const int32_t* cu_seqlens, const hgx_segment* segs,
+                            const int32_t* cu_segs, const int32_t* first_rows, std::string* err) {
+  if (batch > 0 && !first_rows) {
+    *err = "first_rows must be non-null";
+    return HGX_ERR_INVALID_ARG;
+  }
+  std::vector<int32_t> lim;
+  hgx_status st = row_limits(batch, cu_seqlens, segs, cu_segs, &lim, err);
+  if (st != HGX_OK) return st;
+  for (int32_t b = 0; b < batch; ++b) {
+    const int32_t L = cu_seqlens[b + 1] - cu_seqlens[b], f = first_rows[b];
+    if (f < 0 || f > L) {
+      *err = fmt("first row %lld of batch element %lld is outside [0, %lld]", f, b, L);
+      return HGX_ERR_INVALID_ARG;
+    }
+    for (int32_t i = 0; i < f; ++i)
+      if (lim[static_cast<size_t>(cu_seqlens[b] + i)] > f) {
+        *err = fmt("row %lld of batch element %lld is reused but sees key %lld, which is "
+                   "recomputed", i, b, f);
+        return HGX_ERR_INVALID_ARG;
+      }
+  }
+  return HGX_OK;
+}
+
 namespace {
 
 int popcount4(const uint32_t* m) {
@@ -133,9 +158,11 @@ int popcount4(const uint32_t* m) {
 
 hgx_status build_plan(int32_t batch, const int32_t* cu_seqlens, const hgx_segment* segs,
                       const int32_t* cu_segs, int32_t num_kv_heads, Plan* plan,
-                      std::string* err) {
+                      std::string* err, const int32_t* first_rows) {
   hgx_status st = row_limits(batch, cu_seqlens, segs, cu_segs, &plan->lim, err);
   if (st != HGX_OK) return st;
+  if (first_rows && (st = check_first_rows(batch, cu_seqlens, segs, cu_segs, first_rows, err)) != HGX_OK)
+    return st;
   plan->batch = batch;
   plan->total_tokens = batch ? cu_seqlens[batch] : 0;
   plan->items.clear();
@@ -144,7 +171,9 @@ hgx_status build_plan(int32_t batch, const int32_t* cu_seqlens, const hgx_segmen
   plan->hole_masks.clear();
   plan->has_holes = false;
   plan->visible_pairs = 0;
-  for (int32_t x : plan->lim) plan->visible_pairs += static_cast<uint64_t>(x);
+  for (int32_t b = 0; b < batch; ++b)
+    for (int32_t i = first_rows ? first_rows[b] : 0; i < cu_seqlens[b + 1] - cu_seqlens[b]; ++i)
+      plan->visible_pairs += static_cast<uint64_t>(plan->lim[static_cast<size_t>(cu_seqlens[b] + i)]);
   for (int32_t s = 0; batch > 0 && s < cu_segs[batch]; ++s)
     if (segs[s].kind == HGX_SEG_GEN_IMAGE) plan->has_holes = true;
   if (plan->has_holes) plan->hole_base.assign(static_cast<size_t>(plan->total_tokens), -1);
@@ -171,13 +200,14 @@ hgx_status build_plan(int32_t batch, const int32_t* cu_seqlens, const hgx_segmen
           }
           for (int32_t i = sg.start; i < sg.start + sg.len; ++i) {
             plan->hole_base[static_cast<size_t>(base + i)] = mbase;
-            plan->visible_pairs -= static_cast<uint64_t>(hidden);
+            if (!first_rows || i >= first_rows[b]) plan->visible_pairs -= static_cast<uint64_t>(hidden);
           }
         }
         if (sg.kind == HGX_SEG_GEN_IMAGE) gens.emplace_back(sg.start, sg.start + sg.len);
       }
     }
-    for (int32_t r0 = 0; r0 < L; r0 += kBlockTokens) {
+    const int32_t first = first_rows ? first_rows[b] : 0;
+    for (int32_t r0 = first / kBlockTokens * kBlockTokens; r0 < L; r0 += kBlockTokens) {
       const int32_t r1 = std::min(L, r0 + kBlockTokens);
       int32_t lo = INT32_MAX, hi = 0;
       bool holes = false;
@@ -192,6 +222,7 @@ hgx_status build_plan(int32_t batch, const int32_t* cu_seqlens, const hgx_segmen
       it.kv0 = base;
       it.len = L;
       it.list_off = -1;
+      it.first = first;
       if (!holes) {
         it.n_full = lo / kBlockKeys;
         it.n_total = (hi + kBlockKeys - 1) / kBlockKeys;
@@ -244,6 +275,7 @@ void tile_classes(const Plan& plan, int32_t batch, const int32_t* cu_seqlens,
       const WorkItem* it = by_q0[static_cast<size_t>(base + r0)];
       const size_t at = out->size();
       out->resize(at + static_cast<size_t>(nkb), HGX_TILE_SKIP);
+      if (!it) continue;  // query block of a reused prefix: nothing is computed
       if (it->list_off < 0) {
         for (int32_t kb = 0; kb < nkb; ++kb)
           (*out)[at + kb] = kb < it->n_full ? HGX_TILE_FULL : kb < it->n_total ? HGX_TILE_PARTIAL : HGX_TILE_SKIP;
@@ -257,16 +289,22 @@ void tile_classes(const Plan& plan, int32_t batch, const int32_t* cu_seqlens,
   }
 }
 
-void mrope_tables(double theta, int32_t head_dim, const int32_t section[3], double* inv_freq,
-                  int32_t* axis) {
+void mrope_tables(double theta, int32_t head_dim, const int32_t section[3], int32_t layout,
+                  double* inv_freq, int32_t* axis) {
   const int32_t half = head_dim / 2;
   for (int32_t k = 0; k < half; ++k) {
     inv_freq[k] = std::pow(theta, -2.0 * static_cast<double>(k) / static_cast<double>(head_dim));
-    // interleaved: h and w take every third frequency (offsets 1 and 2) while they have
-    // slots left; t takes offset 0 and everything after the interleaved run.
     int32_t a = 0;
-    if (k % 3 == 1 && k < 3 * section[1]) a = 1;
-    else if (k % 3 == 2 && k < 3 * section[2]) a = 2;
+    if (layout == HGX_ROPE_2D_ALTERNATING) {
+      a = k % 2 == 0 ? 2 : 1;  // x (the w column) on even frequencies, y (h) on odd ones
+    } else if (layout == HGX_ROPE_2D_HALVES) {
+      a = k < half / 2 ? 2 : 1;  // x on the first half of the frequencies, y on the second
+    } else {
+      // interleaved: h and w take every third frequency (offsets 1 and 2) while they have
+      // slots left; t takes offset 0 and everything after the interleaved run.
+      if (k % 3 == 1 && k < 3 * section[1]) a = 1;
+      else if (k % 3 == 2 && k < 3 * section[2]) a = 2;
+    }
     axis[k] = a;
   }
 }

@@ -37,7 +37,7 @@ struct WorkItem {
   int32_t n_full;    // prefix form: key blocks [0, n_full) need no compare
   int32_t n_total;   // key blocks to process
   int32_t list_off;  // -1: prefix form; else offset into the key-block list
-  int32_t pad;
+  int32_t first;     // rows before this local row are not written (cached prefix)
 };
 static_assert(sizeof(WorkItem) == 32, "work item layout");
 
@@ -66,19 +66,26 @@ hgx_status validate_descriptor(int32_t batch, const int32_t* cu_seqlens,
 hgx_status row_limits(int32_t batch, const int32_t* cu_seqlens, const hgx_segment* segs,
                       const int32_t* cu_segs, std::vector<int32_t>* lim, std::string* err);
 
-// Validates, computes limits and the sorted work list for num_kv_heads KV heads.
+// Validates, computes limits and the sorted work list for num_kv_heads KV heads. With
+// first_rows (host, [batch], may be NULL) only rows [first_rows[b], L_b) of element b are
+// planned; every earlier row must see no key at or after first_rows[b] (a cached prefix).
 hgx_status build_plan(int32_t batch, const int32_t* cu_seqlens, const hgx_segment* segs,
                       const int32_t* cu_segs, int32_t num_kv_heads, Plan* plan,
-                      std::string* err);
+                      std::string* err, const int32_t* first_rows = nullptr);
+
+// Checks first_rows (host, [batch]) against a valid descriptor: each within [0, L_b] and no
+// row before it seeing a key at or after it. INVALID_ARG with *err otherwise.
+hgx_status check_first_rows(int32_t batch, const int32_t* cu_seqlens, const hgx_segment* segs,
+                            const int32_t* cu_segs, const int32_t* first_rows, std::string* err);
 
 // Tile classes of every (query block, key block) of every batch element in order (after
 // a successful build_plan with the same descriptor).
 void tile_classes(const Plan& plan, int32_t batch, const int32_t* cu_seqlens,
                   std::vector<uint8_t>* out);
 
-// Frequency table of the interleaved mRoPE: inv_freq[k] = theta^(-2k/D) and the axis
-// (0 t, 1 h, 2 w) that drives frequency k.
-void mrope_tables(double theta, int32_t head_dim, const int32_t section[3], double* inv_freq,
-                  int32_t* axis);
+// Frequency table of the rotary embedding: inv_freq[k] = theta^(-2k/D) and the axis
+// (0 t, 1 h, 2 w) that drives frequency k under the given hgx_rope_layout.
+void mrope_tables(double theta, int32_t head_dim, const int32_t section[3], int32_t layout,
+                  double* inv_freq, int32_t* axis);
 
 }  // namespace hgx

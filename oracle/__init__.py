@@ -31,4 +31,6 @@ from .reference import (  # noqa: F401
     forward,
     unmasked_pairs,
     tile_classes,
+    qkv_projection,
+    layer_forward,
 )

@@ -288,3 +288,38 @@ def attention_rows(q, k, v, pos, wq, wk, cu_seqlens, segs, cu_segs, tokens: Sequ
                 p = np.exp(s - s.max())
                 res[n, h] = (p @ vv[:, h // G, :]) / p.sum()
     return res
+
+
+# ---------------------------------------------------------------------------------------
+# The attention layer around the core: QKV projection and output projection
+# ("hidream-o1-p100a" model card, "What this model is": hidden size 4096, GQA 32/8, head
+# 128, so the projection maps 4096 features to 32*128 + 2 * 8*128 = 6144 and back to 4096)
+# ---------------------------------------------------------------------------------------
+def qkv_projection(x, w_qkv, num_q_heads=32, num_kv_heads=8, head_dim=128):
+    """x [T, hidden] @ w_qkv[N, hidden]^T split into q [T,Hq,D], k [T,Hkv,D], v [T,Hkv,D];
+    output columns are ordered q heads, then k heads, then v heads."""
+    y = bf16_to_f64(x) @ bf16_to_f64(w_qkv).T
+    nq, nk = num_q_heads * head_dim, num_kv_heads * head_dim
+    T = y.shape[0]
+    return (y[:, :nq].reshape(T, num_q_heads, head_dim), y[:, nq:nq + nk].reshape(T, num_kv_heads, head_dim),
+            y[:, nq + nk:nq + 2 * nk].reshape(T, num_kv_heads, head_dim))
+
+
+def layer_forward(x, w_qkv, w_o, pos, wq, wk, cu_seqlens, segs, cu_segs, theta=5.0e6, sections=(24, 20, 20),
+                  eps=1e-6, scale=None, layout=ROPE_MROPE_INTERLEAVED):
+    """x -> QKV projection -> q/k RMSNorm + RoPE -> masked GQA attention -> output projection,
+    fp64. Returns (y [T, hidden], attention output [T, Hq, D], q', k', v)."""
+    q, k, v = qkv_projection(x, w_qkv)
+    D = q.shape[-1]
+    phi = mrope_angles(pos, theta, D, sections, layout)
+    qp = rope_rotate_half(rms_norm(q, bf16_to_f64(wq), eps), phi)
+    kp = rope_rotate_half(rms_norm(k, bf16_to_f64(wk), eps), phi)
+    att = np.zeros_like(qp)
+    for b in range(len(cu_seqlens) - 1):
+        t0, t1 = int(cu_seqlens[b]), int(cu_seqlens[b + 1])
+        if t1 > t0:
+            mask = dense_mask(_batch_segments(segs, cu_segs, b), t1 - t0)
+            att[t0:t1] = masked_gqa_attention(qp[t0:t1], kp[t0:t1], v[t0:t1], mask, scale)
+    T = att.shape[0]
+    y = att.reshape(T, -1) @ bf16_to_f64(w_o).T
+    return y, att, qp, kp, v

@@ -286,3 +286,28 @@ def test_prologue_order_norm_then_rotate():
     qp, kp = O.prologue(t["q"][:8], t["k"][:8], pos[:8], t["wq"], t["wk"])
     qn = O.rms_norm(O.bf16_to_f64(t["q"][:8]), O.bf16_to_f64(t["wq"]), 1e-6)
     np.testing.assert_allclose(np.linalg.norm(qp, axis=-1), np.linalg.norm(qn, axis=-1), rtol=1e-12)
+
+
+def test_layer_with_selecting_weights_reduces_to_the_core():
+    """With projection weights that copy input columns (0/1 matrices) the layer is the
+    attention core on those columns, and an identity output projection returns the
+    attention output unchanged: pins the q | k | v column order and both transposes."""
+    rng = np.random.default_rng(21)
+    T, hidden = 12, 4096
+    x = rng.standard_normal((T, hidden))
+    perm = rng.permutation(hidden)
+    w_qkv = np.zeros((6144, hidden))
+    cols = np.concatenate([perm, perm[:2048]])  # q from perm[:4096], k and v from perm[:1024], perm[1024:2048]
+    w_qkv[np.arange(6144), cols] = 1.0
+    w_o = np.eye(4096)
+    pos = np.stack([np.arange(T)] * 3, axis=1)
+    segs = np.array([[0, 5, O.CAUSAL], [5, 7, O.FULL_SEQUENCE]])
+    wq = np.ones(128)
+    y, att, qp, kp, v = O.layer_forward(x, w_qkv, w_o, pos, wq, wq, [0, T], segs, [0, 2])
+    q_in = x[:, perm[:4096]].reshape(T, 32, 128)
+    k_in = x[:, perm[:1024]].reshape(T, 8, 128)
+    v_in = x[:, perm[1024:2048]].reshape(T, 8, 128)
+    ref, qr, kr = O.forward(q_in, k_in, v_in, pos, wq, wq, [0, T], segs, [0, 2])
+    np.testing.assert_allclose(att, ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(y, att.reshape(T, -1), rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(v, v_in)

@@ -470,7 +470,7 @@ def _kernel_sha():
     import hashlib
 
     hsh = hashlib.sha256()
-    for f in ("attention.cu", "sm100.cuh", "kernels.h", "planner.h", "exp2_poly.h"):
+    for f in ("attention.cu", "sm100.cuh", "kernels.h", "planner.h", "exp2_poly.h", "waits.cuh"):
         with open(os.path.join(ROOT, "unified_text_pixel_b200", "csrc", f), "rb") as fh:
             hsh.update(fh.read())
     return hsh.hexdigest()[:16]

@@ -33,4 +33,5 @@ from .reference import (  # noqa: F401
     tile_classes,
     qkv_projection,
     layer_forward,
+    layer_rows,
 )

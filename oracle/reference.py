@@ -323,3 +323,39 @@ def layer_forward(x, w_qkv, w_o, pos, wq, wk, cu_seqlens, segs, cu_segs, theta=5
     T = att.shape[0]
     y = att.reshape(T, -1) @ bf16_to_f64(w_o).T
     return y, att, qp, kp, v
+
+
+def layer_rows(x, w_qkv, w_o, pos, wq, wk, cu_seqlens, segs, cu_segs, tokens: Sequence[int],
+               theta=5.0e6, sections=(24, 20, 20), eps=1e-6, scale=None, layout=ROPE_MROPE_INTERLEAVED):
+    """layer_forward for selected packed tokens only: (y rows [n, hidden], attention rows
+    [n, Hq, D]). Keys and values of the whole batch element are projected; queries only for
+    the selected tokens."""
+    tokens = [int(t) for t in tokens]
+    xf, wqkv = bf16_to_f64(x), bf16_to_f64(w_qkv)
+    pos = np.asarray(pos)
+    cu = [int(c) for c in cu_seqlens]
+    att = np.zeros((len(tokens), 32, 128))
+    for b in range(len(cu) - 1):
+        t0, t1 = cu[b], cu[b + 1]
+        picked = [(n, t) for n, t in enumerate(tokens) if t0 <= t < t1]
+        if not picked:
+            continue
+        kv = xf[t0:t1] @ wqkv[4096:].T
+        k = kv[:, :1024].reshape(-1, 8, 128)
+        v = kv[:, 1024:].reshape(-1, 8, 128)
+        phi_all = mrope_angles(pos[t0:t1], theta, 128, sections, layout)
+        kp = rope_rotate_half(rms_norm(k, bf16_to_f64(wk), eps), phi_all)
+        mask = dense_mask(_batch_segments(segs, cu_segs, b), t1 - t0)
+        sc = 1.0 / np.sqrt(128) if scale is None else scale
+        for n, tok in picked:
+            q = (xf[tok] @ wqkv[:4096].T).reshape(1, 32, 128)
+            qp = rope_rotate_half(rms_norm(q, bf16_to_f64(wq), eps),
+                                  mrope_angles(pos[tok:tok + 1], theta, 128, sections, layout))
+            row = mask[tok - t0]
+            for h in range(32):
+                sv = (kp[:, h // 4, :] @ qp[0, h, :]) * sc
+                sv = np.where(row, sv, -np.inf)
+                pr = np.exp(sv - sv.max())
+                att[n, h] = (pr @ v[:, h // 4, :]) / pr.sum()
+    y = att.reshape(len(tokens), -1) @ bf16_to_f64(w_o).T
+    return y, att

@@ -311,3 +311,16 @@ def test_layer_with_selecting_weights_reduces_to_the_core():
     np.testing.assert_allclose(att, ref, rtol=0, atol=1e-12)
     np.testing.assert_allclose(y, att.reshape(T, -1), rtol=0, atol=1e-12)
     np.testing.assert_array_equal(v, v_in)
+
+
+def test_layer_rows_agrees_with_layer_forward():
+    """The sampled-rows layer oracle used at full size equals the whole-layer oracle."""
+    w = W.custom("small_layer", [[(9, W.CAUSAL), (14, W.FULL_IN_SEGMENT), (6, W.GEN_IMAGE), (5, W.CAUSAL)]], seed=8)
+    lt = W.layer_tensors(w)
+    segs, cu_segs = W.flat_segments(w)
+    pos, cu = W.positions(w), W.cu_seqlens(w)
+    y, att, _, _, _ = O.layer_forward(lt["x"], lt["w_qkv"], lt["w_o"], pos, lt["wq"], lt["wk"], cu, segs, cu_segs)
+    rows = [0, 8, 9, 22, 23, 30, 33]
+    y_r, att_r = O.layer_rows(lt["x"], lt["w_qkv"], lt["w_o"], pos, lt["wq"], lt["wk"], cu, segs, cu_segs, rows)
+    np.testing.assert_allclose(att_r, att[rows], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(y_r, y[rows], rtol=0, atol=1e-11)

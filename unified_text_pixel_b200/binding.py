@@ -53,6 +53,9 @@ _SIGS = {
     "hgx_attn_forward": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_int32] + [ctypes.c_void_p] * 3),
     "hgx_attn_forward_from": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_int32] + [ctypes.c_void_p] * 4),
     "hgx_attn_prologue": (ctypes.c_int, [ctypes.c_void_p] * 7 + [ctypes.c_int32]),
+    "hgx_attn_qkv_projection": (ctypes.c_int, [ctypes.c_void_p] * 10 + [ctypes.c_int32]),
+    "hgx_attn_out_projection": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int32]),
+    "hgx_attn_layer_forward": (ctypes.c_int, [ctypes.c_void_p] * 13 + [ctypes.c_int32] + [ctypes.c_void_p] * 3),
     "hgx_attn_attention": (ctypes.c_int, [ctypes.c_void_p] * 6 + [ctypes.c_int32] + [ctypes.c_void_p] * 3),
     "hgx_attn_row_limits": (ctypes.c_int, [ctypes.c_int32] + [ctypes.c_void_p] * 4 + [ctypes.c_size_t]),
     "hgx_attn_classify": (ctypes.c_int, [ctypes.c_int32] + [ctypes.c_void_p] * 6 + [ctypes.c_size_t, ctypes.c_void_p]),
@@ -202,6 +205,27 @@ class Attention:
                                          _dev_ptr(out), _dev_ptr(pos), _dev_ptr(wq), _dev_ptr(wk), len(cu) - 1,
                                          _ptr(cu), _ptr(sg), _ptr(cs), _ptr(fr))
         self._check(st, "hgx_attn_forward_from")
+
+    def qkv_projection(self, x, w_qkv, q, k, v, pos, wq, wk, stream=None):
+        """q', k', v from x: tcgen05 GEMM with RMSNorm + rotation in its epilogue."""
+        st = lib().hgx_attn_qkv_projection(self._h, _stream_ptr(stream), _dev_ptr(x), _dev_ptr(w_qkv), _dev_ptr(q),
+                                           _dev_ptr(k), _dev_ptr(v), _dev_ptr(pos), _dev_ptr(wq), _dev_ptr(wk),
+                                           int(x.shape[0]))
+        self._check(st, "hgx_attn_qkv_projection")
+
+    def out_projection(self, attn, w_o, y, stream=None):
+        st = lib().hgx_attn_out_projection(self._h, _stream_ptr(stream), _dev_ptr(attn), _dev_ptr(w_o), _dev_ptr(y),
+                                           int(attn.shape[0]))
+        self._check(st, "hgx_attn_out_projection")
+
+    def layer_forward(self, x, w_qkv, w_o, q, k, v, attn, y, pos, wq, wk, cu_seqlens, segs, cu_segs, stream=None):
+        """QKV projection (fused RMSNorm + rotation) -> masked attention -> output projection."""
+        cu, sg, cs = _descriptor(cu_seqlens, segs, cu_segs)
+        st = lib().hgx_attn_layer_forward(self._h, _stream_ptr(stream), _dev_ptr(x), _dev_ptr(w_qkv), _dev_ptr(w_o),
+                                          _dev_ptr(q), _dev_ptr(k), _dev_ptr(v), _dev_ptr(attn), _dev_ptr(y),
+                                          _dev_ptr(pos), _dev_ptr(wq), _dev_ptr(wk), len(cu) - 1, _ptr(cu),
+                                          _ptr(sg), _ptr(cs))
+        self._check(st, "hgx_attn_layer_forward")
 
     def prologue(self, q, k, pos, wq, wk, total_tokens=None, stream=None):
         T = q.shape[0] if total_tokens is None else total_tokens

@@ -9,8 +9,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "libhgx_attn.so")
-SOURCES = ["planner.cpp", "prologue.cu", "attention.cu", "api.cu", "noalloc.cu"]
-HEADERS = ["planner.h", "kernels.h", "sm100.cuh", "exp2_poly.h", os.path.join("..", "..", "include", "hgx_attn.h")]
+SOURCES = ["planner.cpp", "prologue.cu", "attention.cu", "gemm.cu", "api.cu", "noalloc.cu"]
+HEADERS = ["planner.h", "kernels.h", "sm100.cuh", "exp2_poly.h", "waits.cuh", os.path.join("..", "..", "include", "hgx_attn.h")]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall"]

@@ -48,6 +48,9 @@ struct hgx_attn_handle {
   size_t hole_base_cap = 0;
   uint32_t* d_hole_masks = nullptr;
   size_t hole_masks_cap = 0;
+  // (cos, sin) per (token, frequency) for the QKV projection's epilogue
+  void* d_rope_cs = nullptr;
+  size_t rope_cs_cap = 0;
   uint32_t* d_err = nullptr;
   // pinned staging for the plan upload, reused once the previous upload has completed
   uint8_t* h_stage = nullptr;
@@ -101,6 +104,20 @@ bool make_map(CUtensorMap* map, const void* ptr, int heads, int T, int box_heads
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// 2-D bf16 tensor map over a row-major [rows, cols] matrix with a (64, box_rows) box and
+// 128-byte swizzle (the GEMM operands; rows past the end read zeros).
+bool make_map_2d(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols, int box_rows) {
+  PFN_encodeTiled enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 hgx_status ensure_device(hgx_attn_handle* h) {
@@ -265,6 +282,60 @@ hgx_status run_attention(hgx_attn_handle* h, cudaStream_t stream, const void* q,
   return HGX_OK;
 }
 
+hgx_status run_gemm(hgx_attn_handle* h, cudaStream_t stream, const void* a, const void* b,
+                    hgx::GemmParams p) {
+  CUtensorMap ma, mb;
+  if (!make_map_2d(&ma, a, p.M, p.K, 128) || !make_map_2d(&mb, b, p.N, p.K, 256))
+    return fail(h, HGX_ERR_CUDA, "cuTensorMapEncodeTiled failed");
+  p.err = h->d_err;
+  p.wait_limit_ns = h->wait_limit_ns;
+  const int tiles = ((p.M + 127) / 128) * (p.N / 256);
+  const int grid = tiles < h->num_sms ? tiles : h->num_sms;
+  cudaError_t e = hgx::launch_gemm(stream, ma, mb, p, grid);
+  if (e != cudaSuccess) return cuda_fail(h, e, "gemm launch");
+  return HGX_OK;
+}
+
+// QKV projection of total_tokens rows with q/k RMSNorm and rotation in the epilogue.
+hgx_status run_qkv(hgx_attn_handle* h, cudaStream_t stream, const void* x, const void* w_qkv, void* q,
+                   void* k, void* v, const int32_t* pos, const void* wq, const void* wk, int32_t T) {
+  const size_t need = static_cast<size_t>(T) * 64 * sizeof(float2);
+  if (need > h->rope_cs_cap) {
+    if (h->d_rope_cs) cudaFree(h->d_rope_cs);
+    h->d_rope_cs = nullptr;
+    h->rope_cs_cap = 0;
+    if (cudaMalloc(&h->d_rope_cs, need) != cudaSuccess)
+      return fail(h, HGX_ERR_OOM, "cudaMalloc of the rotation table failed");
+    h->rope_cs_cap = need;
+  }
+  cudaError_t e = hgx::launch_rope_table(stream, pos, T, h->rope, h->d_rope_cs);
+  if (e != cudaSuccess) return cuda_fail(h, e, "rotation table launch");
+  hgx::GemmParams p{};
+  p.M = T;
+  p.N = 6144;
+  p.K = 4096;
+  p.mode = 1;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.rope_cs = static_cast<const float2*>(h->d_rope_cs);
+  p.wq = static_cast<const __nv_bfloat16*>(wq);
+  p.wk = static_cast<const __nv_bfloat16*>(wk);
+  p.eps = h->cfg.rms_eps;
+  return run_gemm(h, stream, x, w_qkv, p);
+}
+
+hgx_status run_out_proj(hgx_attn_handle* h, cudaStream_t stream, const void* att, const void* w_o, void* y,
+                        int32_t T) {
+  hgx::GemmParams p{};
+  p.M = T;
+  p.N = 4096;
+  p.K = 4096;
+  p.mode = 0;
+  p.c = y;
+  return run_gemm(h, stream, att, w_o, p);
+}
+
 }  // namespace
 
 extern "C" {
@@ -331,6 +402,7 @@ void hgx_attn_destroy(hgx_attn_handle* h) {
   if (h->d_kblocks) cudaFree(h->d_kblocks);
   if (h->d_hole_base) cudaFree(h->d_hole_base);
   if (h->d_hole_masks) cudaFree(h->d_hole_masks);
+  if (h->d_rope_cs) cudaFree(h->d_rope_cs);
   if (h->d_err) cudaFree(h->d_err);
   if (h->h_stage) cudaFreeHost(h->h_stage);
   if (h->stage_done) cudaEventDestroy(h->stage_done);
@@ -445,6 +517,63 @@ hgx_status hgx_attn_forward_from(hgx_attn_handle* h, void* stream, void* q, void
     if (e != cudaSuccess) return cuda_fail(h, e, "prologue launch");
   }
   if (!h->plan.items.empty() && (st = run_attention(h, s, q, k, v, out)) != HGX_OK) return st;
+  return finish(h, s);
+}
+
+hgx_status hgx_attn_qkv_projection(hgx_attn_handle* h, void* stream, const void* x, const void* w_qkv,
+                                   void* q, void* k, void* v, const int32_t* pos_thw,
+                                   const void* q_norm_w, const void* k_norm_w, int32_t total_tokens) {
+  if (!h) return HGX_ERR_INVALID_ARG;
+  h->last_error.clear();
+  if (total_tokens < 0 || total_tokens > hgx::kMaxTokens)
+    return fail(h, HGX_ERR_INVALID_ARG, "total_tokens out of range");
+  if (total_tokens == 0) return HGX_OK;
+  hgx_status st = check_tensors(h, {x, w_qkv, q, k, v, pos_thw, q_norm_w, k_norm_w});
+  if (st != HGX_OK) return st;
+  if ((st = ensure_device(h)) != HGX_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = run_qkv(h, s, x, w_qkv, q, k, v, pos_thw, q_norm_w, k_norm_w, total_tokens)) != HGX_OK) return st;
+  return finish(h, s);
+}
+
+hgx_status hgx_attn_out_projection(hgx_attn_handle* h, void* stream, const void* attn, const void* w_o,
+                                   void* y, int32_t total_tokens) {
+  if (!h) return HGX_ERR_INVALID_ARG;
+  h->last_error.clear();
+  if (total_tokens < 0 || total_tokens > hgx::kMaxTokens)
+    return fail(h, HGX_ERR_INVALID_ARG, "total_tokens out of range");
+  if (total_tokens == 0) return HGX_OK;
+  hgx_status st = check_tensors(h, {attn, w_o, y});
+  if (st != HGX_OK) return st;
+  if ((st = ensure_device(h)) != HGX_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = run_out_proj(h, s, attn, w_o, y, total_tokens)) != HGX_OK) return st;
+  return finish(h, s);
+}
+
+hgx_status hgx_attn_layer_forward(hgx_attn_handle* h, void* stream, const void* x, const void* w_qkv,
+                                  const void* w_o, void* q, void* k, void* v, void* attn, void* y,
+                                  const int32_t* pos_thw, const void* q_norm_w, const void* k_norm_w,
+                                  int32_t batch, const int32_t* cu_seqlens_host,
+                                  const hgx_segment* segs_host, const int32_t* cu_segs_host) {
+  if (!h) return HGX_ERR_INVALID_ARG;
+  h->last_error.clear();
+  std::string err;
+  int32_t T = 0;
+  hgx_status st = hgx::validate_descriptor(batch, cu_seqlens_host, segs_host, cu_segs_host, &err, &T);
+  if (st != HGX_OK) return fail(h, st, err);
+  if (T == 0) return HGX_OK;
+  if ((st = check_tensors(h, {x, w_qkv, w_o, q, k, v, attn, y, pos_thw, q_norm_w, k_norm_w})) != HGX_OK)
+    return st;
+  const size_t qb = size_t(T) * 8192, kb = size_t(T) * 2048;
+  if (overlaps(attn, qb, q, qb) || overlaps(attn, qb, k, kb) || overlaps(attn, qb, v, kb))
+    return fail(h, HGX_ERR_INVALID_ARG, "attn overlaps q, k or v");
+  if ((st = ensure_device(h)) != HGX_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = prepare_plan(h, s, batch, cu_seqlens_host, segs_host, cu_segs_host)) != HGX_OK) return st;
+  if ((st = run_qkv(h, s, x, w_qkv, q, k, v, pos_thw, q_norm_w, k_norm_w, T)) != HGX_OK) return st;
+  if ((st = run_attention(h, s, q, k, v, attn)) != HGX_OK) return st;
+  if ((st = run_out_proj(h, s, attn, w_o, y, T)) != HGX_OK) return st;
   return finish(h, s);
 }
 

@@ -35,12 +35,14 @@
 #include "exp2_poly.h"
 #include "kernels.h"
 #include "sm100.cuh"
+#include "waits.cuh"
 
 namespace hgx {
 
 namespace {
 
 using namespace sm100;
+using namespace waits;
 
 constexpr int kThreads = 384;
 #ifndef HGX_KV_STAGES
@@ -85,55 +87,6 @@ enum : uint32_t {
   SITE_STALL = 4,
   SITE_DRAIN = 5
 };
-
-struct Ctx {
-  uint32_t bars;           // shared address of barrier 0
-  volatile uint32_t* abort_flag;
-  uint32_t* err;
-  uint64_t limit_ns;
-};
-
-__device__ __forceinline__ uint32_t bar_addr(const Ctx& c, uint32_t i) { return c.bars + 8 * i; }
-
-// Bounded wait for the phase of the given parity. Returns false if the wait ran out (after
-// recording it in the device error word and raising the CTA's abort flag) or if another
-// role already raised the abort flag.
-__device__ __forceinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatile uint32_t* abort_flag,
-                                       uint32_t* err, uint64_t limit_ns, uint32_t site) {
-  uint64_t start = 0;
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if ((it & 63u) == 0) {
-      const uint64_t now = globaltimer_ns();
-      if (start == 0) {
-        start = now;
-      } else if (now - start > limit_ns) {
-        *abort_flag = 1u;
-        atomicOr(err, kErrTimeout | (site << 8));
-        return false;
-      }
-    }
-  }
-}
-
-__device__ __forceinline__ bool wait_bounded(const Ctx& c, uint32_t bar, uint32_t parity,
-                                             uint32_t site) {
-  if (mbar_try_wait(bar, parity)) return true;
-  return wait_slow(bar, parity, c.abort_flag, c.err, c.limit_ns, site);
-}
-
-// Bounded wait that ignores the abort flag: used while draining copies and MMAs that are
-// already in flight, which complete on their own.
-__device__ __forceinline__ void wait_drain(const Ctx& c, uint32_t bar, uint32_t parity) {
-  const uint64_t start = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - start > c.limit_ns) {
-      atomicOr(c.err, kErrTimeout | (SITE_DRAIN << 8));
-      return;
-    }
-  }
-}
 
 // S_X = Q_X K^T over head_dim 128: 8 MMAs of K = 16. Both operands K-major with 128-byte
 // swizzle: rows of 128 B (64 features), 8-row groups 1024 B apart (SBO); features 64..127
@@ -305,8 +258,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // drain: every load this thread issued must land before the CTA exits (on the normal
         // path they all have, and these waits return at once)
         for (int s = 0; s < kStages; ++s)
-          if (loaded & (1u << s)) wait_drain(c, bar_addr(c, BAR_KV_FULL + s), (last_par >> s) & 1u);
-        if (q_loads > 0) wait_drain(c, bar_addr(c, BAR_Q_FULL), (q_loads - 1) & 1u);
+          if (loaded & (1u << s)) wait_drain(c, bar_addr(c, BAR_KV_FULL + s), (last_par >> s) & 1u, SITE_DRAIN);
+        if (q_loads > 0) wait_drain(c, bar_addr(c, BAR_Q_FULL), (q_loads - 1) & 1u, SITE_DRAIN);
       }
       __syncwarp();
     } else if (warp == 1) {
@@ -377,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // every MMA this thread issued must complete before tensor memory is freed
         mma_commit(bar_addr(c, BAR_DRAIN));
-        wait_drain(c, bar_addr(c, BAR_DRAIN), 0);
+        wait_drain(c, bar_addr(c, BAR_DRAIN), 0, SITE_DRAIN);
       }
       __syncwarp();
     }

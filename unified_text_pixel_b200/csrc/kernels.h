@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -42,6 +43,26 @@ size_t attention_smem_bytes();
 cudaError_t launch_attention(cudaStream_t stream, const CUtensorMap& tmap_q,
                              const CUtensorMap& tmap_k, const CUtensorMap& tmap_v,
                              const AttnParams& p, int grid);
+
+struct GemmParams {
+  int32_t M, N, K;           // C[M, N] = A[M, K] * B[N, K]^T; N % 256 == 0, K % 64 == 0
+  int32_t mode;              // 0: C bf16 [M, N]; 1: QKV split with q/k RMSNorm + rotation
+  void* c;                   // mode 0 output
+  void* q;                   // mode 1 outputs: q' [M,32,128], k' [M,8,128], v [M,8,128]
+  void* k;
+  void* v;
+  const float2* rope_cs;     // mode 1: [M, 64] (cos, sin) of every (token, frequency)
+  const __nv_bfloat16* wq;   // mode 1: RMSNorm weights [128]
+  const __nv_bfloat16* wk;
+  float eps;
+  uint32_t* err;
+  uint64_t wait_limit_ns;
+};
+
+cudaError_t launch_gemm(cudaStream_t stream, const CUtensorMap& tmap_a, const CUtensorMap& tmap_b,
+                        const GemmParams& p, int grid);
+cudaError_t launch_rope_table(cudaStream_t stream, const int32_t* pos, int32_t T,
+                              const RopeTables& tab, void* cs);
 
 // Device error word bits written by the attention kernel.
 constexpr uint32_t kErrTimeout = 1u;

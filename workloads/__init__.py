@@ -248,3 +248,22 @@ def custom(name: str, batches: Sequence[Sequence[Tuple[int, int]]], seed: int = 
     for b in batches:
         out.append(_segments([(n, kd, None if kd == CAUSAL else (1, n)) for n, kd in b]))
     return Workload(name, tuple(out), seed=seed, style="hunyuan")
+
+
+def layer_tensors(w: Workload, device: str = "cpu"):
+    """Seeded bf16 inputs of the whole attention layer: dict(x [T, 4096] ~ N(0, 1),
+    w_qkv [6144, 4096] and w_o [4096, 4096] ~ N(0, 1/4096), wq, wk = 1 + N(0, 0.1)), drawn
+    from torch.Generator().manual_seed(seed + 1000) in that order."""
+    g = torch.Generator().manual_seed(w.seed + 1000)
+    T = w.total_tokens
+    hidden = NUM_Q_HEADS * HEAD_DIM
+    nqkv = hidden + 2 * NUM_KV_HEADS * HEAD_DIM
+    x = torch.randn(T, hidden, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    w_qkv = (torch.randn(nqkv, hidden, generator=g, dtype=torch.float32) / hidden ** 0.5).to(torch.bfloat16)
+    w_o = (torch.randn(hidden, hidden, generator=g, dtype=torch.float32) / hidden ** 0.5).to(torch.bfloat16)
+    wq = (1.0 + 0.1 * torch.randn(HEAD_DIM, generator=g, dtype=torch.float32)).to(torch.bfloat16)
+    wk = (1.0 + 0.1 * torch.randn(HEAD_DIM, generator=g, dtype=torch.float32)).to(torch.bfloat16)
+    out = dict(x=x, w_qkv=w_qkv, w_o=w_o, wq=wq, wk=wk)
+    if device != "cpu":
+        out = {n: t.to(device) for n, t in out.items()}
+    return out

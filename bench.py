@@ -452,6 +452,112 @@ def run_gpu(args):
     return 0
 
 
+def run_gpu_layer(args):
+    """--layer: one step is the whole attention layer (QKV projection with fused RMSNorm +
+    rotation, masked attention, output projection), each kernel timed on its own."""
+    import torch
+
+    import unified_text_pixel_b200 as H
+
+    ws, rank, local = _dist_env()
+    torch.cuda.set_device(local)
+    dist = None
+    if ws > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    w = _workload(args.workload)
+    cu, segs, cu_segs = _descriptor(w)
+    T = w.total_tokens
+    att_flops = _visible_pairs(w) * FLOP_PER_PAIR
+    qkv_flops = 2 * T * 4096 * 6144
+    out_flops = 2 * T * 4096 * 4096
+    flops = att_flops + qkv_flops + out_flops
+    lt = W.layer_tensors(w)
+    x_bytes = T * 4096 * 2
+    n_sets = int(min(args.warmup + args.steps, max(8, SET_BUDGET_BYTES // x_bytes)))
+    x0 = lt["x"].cuda()
+    xs = [x0] + [x0.clone() for _ in range(n_sets - 1)]
+    w_qkv, w_o = lt["w_qkv"].cuda(), lt["w_o"].cuda()
+    wq, wk = lt["wq"].cuda(), lt["wk"].cuda()
+    pos = torch.from_numpy(W.positions(w)).cuda()
+    q = torch.empty(T, 32, 128, dtype=torch.bfloat16, device="cuda")
+    k = torch.empty(T, 8, 128, dtype=torch.bfloat16, device="cuda")
+    v = torch.empty(T, 8, 128, dtype=torch.bfloat16, device="cuda")
+    att = torch.empty(T, 32, 128, dtype=torch.bfloat16, device="cuda")
+    y = torch.empty(T, 4096, dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream()
+    a = H.Attention()
+    _log(f"layer {w.name}: T={T}, {flops / 1e9:.1f} GFLOP per step ({qkv_flops / 1e9:.1f} qkv, "
+         f"{att_flops / 1e9:.1f} attention, {out_flops / 1e9:.1f} out), {n_sets} input sets")
+
+    def step(i, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        a.qkv_projection(xs[i % n_sets], w_qkv, q, k, v, pos, wq, wk, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        a.attention(q, k, v, att, cu, segs, cu_segs, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        a.out_projection(att, w_o, y, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for i in range(args.warmup):
+        step(i)
+    if a.sync_status(stream) != H.HGX_OK:
+        raise RuntimeError(a.last_error())
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            step(args.warmup + i, evs[i])
+        stop.record(stream)
+        torch.cuda.synchronize()
+    if a.sync_status(stream) != H.HGX_OK:
+        raise RuntimeError(a.last_error())
+    elapsed_ms = max_over_ranks(start.elapsed_time(stop), dist, "cuda")
+    ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / args.steps for i in range(3)]
+    peaks, peak_src = _peaks()
+    peak = peaks["bf16_tflops"]
+    roof = lambda f, t: {"achieved": f / (t * 1e-3) / 1e12, "frac": f / (t * 1e-3) / 1e12 / peak}  # noqa: E731
+    line = {
+        "metric": "attention-layer TFLOP/s (projection FLOPs + unmasked attention FLOPs)",
+        "value": whole_job_tflops(flops, args.steps, ws, elapsed_ms),
+        "unit": "TFLOP/s",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": elapsed_ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (random-init projection weights)",
+        "config": dict(_config_dict(w, _visible_pairs(w)), layer_gflop_per_step=round(flops / 1e9, 3),
+                       l2=f"inputs larger than L2: a distinct {x_bytes / 1e6:.0f} MB x per step"),
+        "kernel_ms": {"qkv_projection": ms[0], "attention": ms[1], "out_projection": ms[2]},
+        "roofline": dict(bound="tensor", kernel="attention_kernel", unit="TFLOP/s", peak=peak, traffic=None,
+                         peak_source=f"{peak_src} bf16 dense (burst)", **roof(att_flops, ms[1])),
+        "gemm_roofline": {"qkv_projection": roof(qkv_flops, ms[0]), "out_projection": roof(out_flops, ms[2])},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk.summary(),
+    }
+    a.close()
+    if dist:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def _recorded_traffic(name):
     """DRAM bytes per attention launch from the committed ncu summary of this workload, if
     the kernel has not changed since it was taken (the summary records the source hash)."""
@@ -486,6 +592,8 @@ def main():
     p.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the CPU-baseline leg")
     p.add_argument("--ref-step-seconds", type=float, default=4.0, help="oracle seconds per reference step")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--layer", action="store_true",
+                   help="time the whole attention layer (QKV projection, attention, output projection)")
     p.add_argument("--reuse-prefix", action="store_true",
                    help="denoising step that reuses the causal text before <|tms|> (hgx_attn_forward_from)")
     args = p.parse_args()
@@ -493,6 +601,8 @@ def main():
         p.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.layer:
+        return run_gpu_layer(args)
     return run_gpu(args)
 
 

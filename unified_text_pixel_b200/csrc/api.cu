@@ -48,6 +48,8 @@ struct hgx_attn_handle {
   size_t hole_base_cap = 0;
   uint32_t* d_hole_masks = nullptr;
   size_t hole_masks_cap = 0;
+  int32_t* d_cta_offsets = nullptr;  // the persistent CTAs' item lists
+  size_t cta_offsets_cap = 0;
   // (cos, sin) per (token, frequency) for the QKV projection's epilogue
   void* d_rope_cs = nullptr;
   size_t rope_cs_cap = 0;
@@ -170,6 +172,7 @@ hgx_status prepare_plan(hgx_attn_handle* h, cudaStream_t stream, int32_t batch,
     hgx_status st =
         hgx::build_plan(batch, cu, segs, cu_segs, h->cfg.num_kv_heads, &plan, &err, first);
     if (st != HGX_OK) return fail(h, st, err);
+    hgx::assign_ctas(&plan, h->num_sms);
     h->plan = std::move(plan);
     h->key_batch = batch;
     h->key_cu.assign(cu, cu + batch + 1);
@@ -199,6 +202,8 @@ hgx_status prepare_plan(hgx_attn_handle* h, cudaStream_t stream, int32_t batch,
        pl.hole_base.size() * sizeof(int32_t)},
       {reinterpret_cast<void**>(&h->d_hole_masks), &h->hole_masks_cap, pl.hole_masks.data(),
        pl.hole_masks.size() * sizeof(uint32_t)},
+      {reinterpret_cast<void**>(&h->d_cta_offsets), &h->cta_offsets_cap, pl.cta_offsets.data(),
+       pl.cta_offsets.size() * sizeof(int32_t)},
   };
   size_t need = 0;
   for (const Upload& u : up) {
@@ -266,6 +271,7 @@ hgx_status run_attention(hgx_attn_handle* h, cudaStream_t stream, const void* q,
   hgx::AttnParams p{};
   p.items = h->d_items;
   p.n_items = static_cast<int32_t>(h->plan.items.size());
+  p.cta_offsets = h->d_cta_offsets;
   p.total_tokens = T;
   p.lim = h->d_lim;
   p.kblocks = h->plan.has_holes ? h->d_kblocks : nullptr;
@@ -276,8 +282,7 @@ hgx_status run_attention(hgx_attn_handle* h, cudaStream_t stream, const void* q,
   p.flags = h->flags;
   p.err = h->d_err;
   p.wait_limit_ns = h->wait_limit_ns;
-  const int grid = p.n_items < h->num_sms ? p.n_items : h->num_sms;
-  cudaError_t e = hgx::launch_attention(stream, mq, mk, mv, p, grid);
+  cudaError_t e = hgx::launch_attention(stream, mq, mk, mv, p, h->plan.grid);
   if (e != cudaSuccess) return cuda_fail(h, e, "attention launch");
   return HGX_OK;
 }
@@ -402,6 +407,7 @@ void hgx_attn_destroy(hgx_attn_handle* h) {
   if (h->d_kblocks) cudaFree(h->d_kblocks);
   if (h->d_hole_base) cudaFree(h->d_hole_base);
   if (h->d_hole_masks) cudaFree(h->d_hole_masks);
+  if (h->d_cta_offsets) cudaFree(h->d_cta_offsets);
   if (h->d_rope_cs) cudaFree(h->d_rope_cs);
   if (h->d_err) cudaFree(h->d_err);
   if (h->h_stage) cudaFreeHost(h->h_stage);

@@ -152,6 +152,17 @@ __device__ __forceinline__ void exp_store_p(const float (&s)[128], float sl2, fl
   f2_unpack(acc[1], l4[2], l4[3]);
 }
 
+// The CTA's items: a contiguous list from the host's assignment, or a grid-stride walk.
+__device__ __forceinline__ int first_item(const AttnParams& p) {
+  return p.cta_offsets ? p.cta_offsets[blockIdx.x] : static_cast<int>(blockIdx.x);
+}
+__device__ __forceinline__ int end_item(const AttnParams& p) {
+  return p.cta_offsets ? p.cta_offsets[blockIdx.x + 1] : p.n_items;
+}
+__device__ __forceinline__ int next_item(const AttnParams& p, int w) {
+  return p.cta_offsets ? w + 1 : w + static_cast<int>(gridDim.x);
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tmap_q,
                      const __grid_constant__ CUtensorMap tmap_k,
@@ -217,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t pos = 0, qe_par = 0, q_loads = 0;
         uint32_t loaded = 0, last_par = 0;  // per slot: ever loaded, parity of its last load
         bool ok = true;
-        for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
+        for (int w = first_item(p); ok && w < end_item(p); w = next_item(p, w)) {
           const WorkItem it = p.items[w];
           if (q_loads > 0) {
             ok = wait_bounded(c, bar_addr(c, BAR_Q_EMPTY), qe_par, SITE_PRODUCER);
@@ -286,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           return true;
         };
-        for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
+        for (int w = first_item(p); ok && w < end_item(p); w = next_item(p, w)) {
           const WorkItem it = p.items[w];
           const int n = it.n_total;
           if (!(ok = wait_bounded(c, bar_addr(c, BAR_Q_FULL), qf_par, SITE_MMA))) break;
@@ -355,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     if ((p.flags & HGX_DEBUG_STALL_TEST) && x == 0)
       ok = __all_sync(0xffffffffu, wait_bounded(c, bar_addr(c, BAR_STALL), 0, SITE_STALL));
-    for (int w = blockIdx.x; ok && w < p.n_items; w += gridDim.x) {
+    for (int w = first_item(p); ok && w < end_item(p); w = next_item(p, w)) {
       const WorkItem it = p.items[w];
       const int32_t tok = it.q0 + 32 * x + (row >> 2);
       const int32_t head = 4 * it.g + (row & 3);

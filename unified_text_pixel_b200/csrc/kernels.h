@@ -25,6 +25,8 @@ cudaError_t launch_prologue(cudaStream_t stream, void* q, void* k, const int32_t
 struct AttnParams {
   const WorkItem* items;
   int32_t n_items;
+  const int32_t* cta_offsets;  // CTA c takes items [cta_offsets[c], cta_offsets[c+1]);
+                               // NULL: CTA c takes items c, c + gridDim.x, ...
   int32_t total_tokens;
   const int32_t* lim;      // [T] exclusive key limit per packed row, local
   const uint32_t* kblocks;     // key-block lists of list-form items (holes only)

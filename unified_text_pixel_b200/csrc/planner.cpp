@@ -16,6 +16,8 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdio>
+#include <functional>
+#include <queue>
 
 namespace hgx {
 
@@ -259,6 +261,36 @@ hgx_status build_plan(int32_t batch, const int32_t* cu_seqlens, const hgx_segmen
   std::stable_sort(plan->items.begin(), plan->items.end(),
                    [](const WorkItem& a, const WorkItem& b) { return a.n_total > b.n_total; });
   return HGX_OK;
+}
+
+void assign_ctas(Plan* plan, int32_t ctas) {
+  const int32_t n = static_cast<int32_t>(plan->items.size());
+  const int32_t g = std::max(1, std::min(ctas, n));
+  plan->grid = n ? g : 0;
+  plan->cta_offsets.assign(static_cast<size_t>(g) + 1, 0);
+  if (!n) return;
+  // items are sorted by n_total, longest first; the per-item overhead stands for loading Q
+  // and writing O (about two key blocks of work)
+  constexpr int64_t kItemOverhead = 2;
+  using Load = std::pair<int64_t, int32_t>;  // (load, cta)
+  std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+  for (int32_t c = 0; c < g; ++c) heap.push({0, c});
+  std::vector<int32_t> owner(static_cast<size_t>(n));
+  std::vector<int32_t> count(static_cast<size_t>(g), 0);
+  for (int32_t i = 0; i < n; ++i) {
+    Load l = heap.top();
+    heap.pop();
+    owner[static_cast<size_t>(i)] = l.second;
+    ++count[static_cast<size_t>(l.second)];
+    l.first += plan->items[static_cast<size_t>(i)].n_total + kItemOverhead;
+    heap.push(l);
+  }
+  for (int32_t c = 0; c < g; ++c) plan->cta_offsets[static_cast<size_t>(c) + 1] = plan->cta_offsets[static_cast<size_t>(c)] + count[static_cast<size_t>(c)];
+  std::vector<WorkItem> ordered(static_cast<size_t>(n));
+  std::vector<int32_t> at(plan->cta_offsets.begin(), plan->cta_offsets.end() - 1);
+  for (int32_t i = 0; i < n; ++i)  // stable: each CTA keeps the longest-first order
+    ordered[static_cast<size_t>(at[static_cast<size_t>(owner[static_cast<size_t>(i)])]++)] = plan->items[static_cast<size_t>(i)];
+  plan->items.swap(ordered);
 }
 
 void tile_classes(const Plan& plan, int32_t batch, const int32_t* cu_seqlens,

@@ -55,6 +55,10 @@ struct Plan {
   std::vector<int32_t> hole_base;  // [T] first mask index of the row's segment, or -1
   std::vector<uint32_t> hole_masks;  // 4 words per (segment, key block): keys hidden
   bool has_holes = false;
+  // Assignment of the items to the persistent CTAs (assign_ctas): CTA c processes items
+  // [cta_offsets[c], cta_offsets[c + 1]) of `items`, longest first.
+  int32_t grid = 0;
+  std::vector<int32_t> cta_offsets;
 };
 
 // Checks the packed-varlen descriptor. On failure returns INVALID_ARG with *err set.
@@ -77,6 +81,12 @@ hgx_status build_plan(int32_t batch, const int32_t* cu_seqlens, const hgx_segmen
 // row before it seeing a key at or after it. INVALID_ARG with *err otherwise.
 hgx_status check_first_rows(int32_t batch, const int32_t* cu_seqlens, const hgx_segment* segs,
                             const int32_t* cu_segs, const int32_t* first_rows, std::string* err);
+
+// Distributes plan->items over `ctas` persistent CTAs (longest-processing-time first: each
+// item, in decreasing cost, goes to the least loaded CTA; cost = key blocks + a per-item
+// overhead), reorders the items so that every CTA's list is contiguous, and sets grid and
+// cta_offsets. grid = min(ctas, number of items).
+void assign_ctas(Plan* plan, int32_t ctas);
 
 // Tile classes of every (query block, key block) of every batch element in order (after
 // a successful build_plan with the same descriptor).

@@ -244,3 +244,30 @@ def test_binding_raises_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(B, "_lib", None)
     with pytest.raises(B.HgxError):
         B.lib()
+
+
+def _noalloc_status(cfg, cu, segs, cu_segs):
+    L = B.lib()
+    fn = L.hgx_attn_forward_noalloc
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.c_void_p] * 9 + [ctypes.c_int32] + [ctypes.c_void_p] * 3 + [ctypes.c_int32]
+    cu, sg, cs = B._descriptor(cu, segs, cu_segs)
+    z = [ctypes.c_void_p(0x40000000 * (i + 1)) for i in range(7)]
+    return fn(ctypes.byref(cfg), None, *z, len(cu) - 1, B._ptr(cu), B._ptr(sg), B._ptr(cs), 1)
+
+
+def test_noalloc_rejects_before_device_work():
+    """The allocation-free entry point checks its fixed limits and the descriptor on the
+    host: too many tokens or a gen_image segment -> UNSUPPORTED, malformed -> INVALID_ARG."""
+    cfg = B.Attention.default_config()
+    assert _noalloc_status(cfg, [0, 16385], [[0, 16385, 0]], [0, 1]) == B.HGX_ERR_UNSUPPORTED
+    assert _noalloc_status(cfg, [0, 10], [[0, 4, 0], [4, 6, 3]], [0, 2]) == B.HGX_ERR_UNSUPPORTED
+    assert _noalloc_status(cfg, [0, 10], [[0, 4, 0], [5, 5, 1]], [0, 2]) == B.HGX_ERR_INVALID_ARG
+    bad = B.Attention.default_config()
+    bad.num_q_heads = 16
+    assert _noalloc_status(bad, [0, 10], [[0, 10, 0]], [0, 1]) == B.HGX_ERR_UNSUPPORTED
+    bad = B.Attention.default_config()
+    bad.rope_layout = 7
+    assert _noalloc_status(bad, [0, 10], [[0, 10, 0]], [0, 1]) == B.HGX_ERR_INVALID_ARG
+    # an empty batch is done without touching the device
+    assert _noalloc_status(cfg, [0], np.zeros((0, 3)), [0]) == B.HGX_OK

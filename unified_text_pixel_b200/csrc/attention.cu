@@ -44,7 +44,22 @@ namespace {
 using namespace sm100;
 using namespace waits;
 
-constexpr int kThreads = 384;
+#ifndef HGX_SOFTMAX_SPLIT
+#define HGX_SOFTMAX_SPLIT 1
+#endif
+// Softmax warps per row of a tile: 1 -- one thread holds a whole 128-column row; 2 -- two
+// warps on the same tensor-memory lanes each take 64 columns (twice the softmax warps,
+// half the dependent work per warp; the row maximum is exchanged through shared memory).
+// Both give the same results within rounding; on B200 split 2 measured no faster (within
+// 1% at 8k-16k tokens, 5% slower at 1k), so 1 is the default.
+constexpr int kSplit = HGX_SOFTMAX_SPLIT;
+static_assert(kSplit == 1 || kSplit == 2, "softmax split");
+constexpr int kCols = 128 / kSplit;               // score columns per softmax thread
+constexpr int kSoftmaxThreads = 128 * kSplit;     // per tile
+constexpr int kThreads = 128 + 2 * kSoftmaxThreads;
+// register budgets after setmaxnreg (launch: 384 x 168 or 640 x 96 registers)
+constexpr uint32_t kRegsLow = kSplit == 1 ? 120 : 64;   // producer/MMA warpgroup
+constexpr uint32_t kRegsHigh = kSplit == 1 ? 192 : 104;  // softmax warpgroups
 #ifndef HGX_KV_STAGES
 #define HGX_KV_STAGES 4
 #endif
@@ -69,7 +84,11 @@ enum : uint32_t {
   BAR_COUNT = BAR_DRAIN + 1
 };
 constexpr uint32_t kMiscOffset = kBarOffset + 8 * BAR_COUNT;  // tmem base, abort flag
-constexpr uint32_t kSmemUsed = kMiscOffset + 16;
+// row-maximum / row-sum exchange between the two halves of a row (kSplit == 2):
+// [iteration parity][tile][half][row] floats
+constexpr uint32_t kXchgOffset = kMiscOffset + 16;
+constexpr uint32_t kXchgBytes = kSplit == 2 ? 2 * 2 * 2 * 128 * 4 : 0;
+constexpr uint32_t kSmemUsed = kXchgOffset + kXchgBytes;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // slack to align the base to 1024 B
 
 constexpr uint32_t kTmemCols = 512;
@@ -92,7 +111,7 @@ enum : uint32_t {
 // swizzle: rows of 128 B (64 features), 8-row groups 1024 B apart (SBO); features 64..127
 // sit in the second 16 KB half of the tile.
 __device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint32_t q_tile, uint32_t k_tile) {
-#pragma unroll
+#pragma unroll 1
   for (int kk = 0; kk < 8; ++kk) {
     const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
     const uint64_t a = smem_desc_sw128(q_tile + off, 16, 1024);
@@ -106,7 +125,7 @@ __device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint32_t q_tile, uint3
 // 8-key groups 1024 B apart (SBO), the two 64-feature halves 16 KB apart (LBO).
 __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_tile,
                                          bool accumulate) {
-#pragma unroll
+#pragma unroll 1
   for (int kk = 0; kk < 8; ++kk) {
     const uint64_t b = smem_desc_sw128(v_tile + kk * 2048, kHalfBytes, 1024);
     mma_ts(tmem_o, tmem_p + kk * 8, b, kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
@@ -123,14 +142,14 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint3
 // P over the first 64 columns of S (key 2c in the low half of column c). Scale-and-shift
 // and the row sum run as paired fp32 instructions; the row sum is kept in 4 partial sums
 // (two pairs) returned in l4.
-template <bool kPoly>
-__device__ __forceinline__ void exp_store_p(const float (&s)[128], float sl2, float mb,
+template <bool kPoly, int N>
+__device__ __forceinline__ void exp_store_p(const float (&s)[N], float sl2, float mb,
                                             uint32_t tS, float (&l4)[4]) {
   const uint64_t scale2 = f2_pack(sl2, sl2);
   const uint64_t shift2 = f2_pack(-mb, -mb);
   uint64_t acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
-  for (int q4 = 0; q4 < 4; ++q4) {  // 32 keys -> 16 packed columns at a time
+  for (int q4 = 0; q4 < N / 32; ++q4) {  // 32 keys -> 16 packed columns at a time
     uint32_t pk[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
@@ -190,9 +209,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(bar_addr(c, BAR_S_FULL + x), 1);
-      mbar_init(bar_addr(c, BAR_P_FULL + x), 128);
+      mbar_init(bar_addr(c, BAR_P_FULL + x), kSoftmaxThreads);
       mbar_init(bar_addr(c, BAR_O_FULL + x), 1);
-      mbar_init(bar_addr(c, BAR_O_EMPTY + x), 128);
+      mbar_init(bar_addr(c, BAR_O_EMPTY + x), kSoftmaxThreads);
     }
     mbar_init(bar_addr(c, BAR_STALL), 1);
     mbar_init(bar_addr(c, BAR_DRAIN), 1);
@@ -209,16 +228,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  // Registers: launched at 168 per thread (384 x 168 = 64512). The producer/MMA warpgroup
-  // hands registers to the two softmax warpgroups: 128 x 120 + 256 x 192 = 64512, the
-  // split at which neither side spills. Only that warpgroup releases and only the softmax
+  // Registers (one warp per row): launched at 168 per thread (384 x 168 = 64512). The
+  // producer/MMA warpgroup hands registers to the two softmax warpgroups: 128 x 120 +
+  // 256 x 192 = 64512, the split at which neither side spills. (Two warps per row: 640
+  // threads at 96 registers each, no hand-over.) Only that warpgroup releases and only the softmax
   // warpgroups take, exactly the same amount, so no increase can wait on a warp that is
   // itself waiting; no budget is ever restored (a warp that took back registers early
   // could starve a softmax warp's increase for good). Each role ends in its own branch
   // at a named barrier over all threads, so no code runs under two budgets, and the waits
   // are inlined (a called function cannot serve regions with different budgets).
   if (warp < 4) {
-    regs_decrease<120>();
+    if constexpr (kRegsLow != kRegsHigh) regs_decrease<kRegsLow>();
     if (warp == 0) {
       // ------------------------------------------------------------------ TMA producer
       if (lane == 0) {
@@ -353,19 +373,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_dealloc(tmem, kTmemCols);
     }
   } else {
-    regs_increase<192>();
+    if constexpr (kRegsLow != kRegsHigh) regs_increase<kRegsHigh>();
     // ------------------------------------------------------------------ softmax
-    const int x = (warp - 4) >> 2;      // tile
-    const int quarter = warp & 3;       // tensor-memory lanes 32*quarter .. +31
+    const int x = (warp - 4) / (4 * kSplit);     // tile
+    const int half = ((warp - 4) >> 2) % kSplit;  // which kCols columns of the row
+    const int quarter = warp & 3;                // tensor-memory lanes 32*quarter .. +31
     const int row = quarter * 32 + lane;
     const uint32_t lane_bits = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_bits + col_s(x);
-    const uint32_t tO = tmem + lane_bits + col_o(x);
+    const uint32_t tS = tmem + lane_bits + col_s(x) + kCols * half;      // S columns
+    const uint32_t tP = tmem + lane_bits + col_s(x) + kCols / 2 * half;  // P columns
+    const uint32_t tO = tmem + lane_bits + col_o(x) + kCols * half;      // O columns
+    float* xchg = reinterpret_cast<float*>(gbase + kXchgOffset);
     const float sl2 = p.scale_log2;
     uint32_t s_par = 0, o_par = 0;
+    int xpar = 0;  // exchange buffer parity
+    // one decision for every thread of the tile: its two halves must leave together
+    auto agree = [&](bool v) {
+      if constexpr (kSplit == 1) return __all_sync(0xffffffffu, v);
+      else return named_bar_and(2 + x, kSoftmaxThreads, v);
+    };
     bool ok = true;
     if ((p.flags & HGX_DEBUG_STALL_TEST) && x == 0)
-      ok = __all_sync(0xffffffffu, wait_bounded(c, bar_addr(c, BAR_STALL), 0, SITE_STALL));
+      ok = agree(wait_bounded(c, bar_addr(c, BAR_STALL), 0, SITE_STALL));
     for (int w = first_item(p); ok && w < end_item(p); w = next_item(p, w)) {
       const WorkItem it = p.items[w];
       const int32_t tok = it.q0 + 32 * x + (row >> 2);
@@ -383,47 +412,72 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint4 hm = make_uint4(0u, 0u, 0u, 0u);
         if (!full && hbase >= 0)
           hm = *reinterpret_cast<const uint4*>(p.hole_masks + 4 * static_cast<size_t>(hbase + kb));
-        ok = __all_sync(0xffffffffu, wait_bounded(c, bar_addr(c, BAR_S_FULL + x), s_par,
-                                                   SITE_SOFTMAX));
-        if (!ok) break;
+        bool got = wait_bounded(c, bar_addr(c, BAR_S_FULL + x), s_par, SITE_SOFTMAX);
+        if constexpr (kSplit == 1) {
+          if (!(ok = __all_sync(0xffffffffu, got))) break;
+        }
         s_par ^= 1u;
         tc_fence_after();
-        uint32_t sr[4][32];
+        // (with two halves an aborted wait still loads: tensor memory is always readable,
+        // and the tile decides together at the exchange below)
+        uint32_t sr[kCols / 32][32];
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) tmem_ld32(tS + 32 * ch, sr[ch]);
+        for (int ch = 0; ch < kCols / 32; ++ch) tmem_ld32(tS + 32 * ch, sr[ch]);
         tmem_wait_ld();
-        float s[128];
+        float s[kCols];
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch)
+        for (int ch = 0; ch < kCols / 32; ++ch)
 #pragma unroll
           for (int e = 0; e < 32; ++e) s[32 * ch + e] = __uint_as_float(sr[ch][e]);
         if (!full) {
-          const int nvis = row_lim - 128 * kb;  // keys [0, nvis) of this block are in the prefix
+          // keys [0, nvis) of this block are in the prefix
+          const int nvis = row_lim - 128 * kb - kCols * half;
           if (hbase >= 0) {
-            const uint32_t hw[4] = {hm.x, hm.y, hm.z, hm.w};  // keys hidden by Gen Image holes
+            // keys hidden by Gen Image holes: the mask words of this thread's columns, picked
+            // up front so that every index below is a compile-time constant
+            uint32_t hw[kCols / 32];
+            if constexpr (kSplit == 1) {
+              hw[0] = hm.x; hw[1] = hm.y; hw[2 % (kCols / 32)] = hm.z; hw[3 % (kCols / 32)] = hm.w;
+            } else {
+              hw[0] = half ? hm.z : hm.x;
+              hw[1] = half ? hm.w : hm.y;
+            }
 #pragma unroll
-            for (int e = 0; e < 128; ++e)
+            for (int e = 0; e < kCols; ++e)
               if (e >= nvis || ((hw[e >> 5] >> (e & 31)) & 1u)) s[e] = -INFINITY;
           } else {
 #pragma unroll
-            for (int e = 0; e < 128; ++e)
+            for (int e = 0; e < kCols; ++e)
               if (e >= nvis) s[e] = -INFINITY;
           }
         }
-        // row max: 8 independent chains of 16 scores (three-input max), then a tree; a
-        // single 128-long chain would expose its whole latency with one softmax warp per
-        // scheduler
-        float m8[8];
+        // row max: independent chains of 16 scores (three-input max), then a tree; a single
+        // long chain would expose its whole latency
+        float m8[kCols / 16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < kCols / 16; ++i) {
           const float* c16 = s + 16 * i;
           float m = fmax3(c16[0], c16[1], c16[2]);
 #pragma unroll
           for (int e = 3; e < 15; e += 2) m = fmax3(m, c16[e], c16[e + 1]);
           m8[i] = fmaxf(m, c16[15]);
         }
-        const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]),
-                               fmaxf(m8[6], m8[7]));
+        float mx = m8[0];
+#pragma unroll
+        for (int i = 1; i < kCols / 16; ++i) mx = fmaxf(mx, m8[i]);
+        if constexpr (kSplit == 2) {
+          // exchange with the other half of the row; the barrier also decides, for the
+          // whole tile, whether every wait succeeded
+          float* slot = xchg + ((xpar * 2 + x) * 2) * 128;
+          slot[half * 128 + row] = mx;
+          // the barrier also orders this half's S loads before the other half's P stores,
+          // which overwrite S columns 32..63 of the tile
+          tc_fence_before();
+          if (!(ok = named_bar_and(2 + x, kSoftmaxThreads, got))) break;
+          tc_fence_after();
+          mx = fmaxf(mx, slot[(half ^ 1) * 128 + row]);
+          xpar ^= 1;
+        }
         const float m_new = fmaxf(m_used, mx);
         float alpha = 1.f;
         bool rescale = false;
@@ -432,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else if (__any_sync(0xffffffffu, (m_new - m_used) * sl2 > 8.0f)) {
           // warp-uniform: the tensor-memory loads and stores of the O rescale are
           // warp-collective, so when any row of the warp needs it every row rescales (by
-          // its own factor <= 1)
+          // its own factor <= 1); both halves of a row see the same maxima, so they agree
           alpha = ex2_approx((m_used - m_new) * sl2);
           m_used = m_new;
           rescale = true;
@@ -443,15 +497,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float mb = m_used == -INFINITY ? 0.f : m_used * sl2;
         float l4[4];
         if (full)
-          exp_store_p<true>(s, sl2, mb, tS, l4);   // no -inf here: the polynomial may be used
+          exp_store_p<true, kCols>(s, sl2, mb, tP, l4);   // no -inf here: polynomial allowed
         else
-          exp_store_p<false>(s, sl2, mb, tS, l4);  // masked scores: MUFU gives exact zeros
+          exp_store_p<false, kCols>(s, sl2, mb, tP, l4);  // masked scores: MUFU gives zeros
         l = fmaf(l, alpha, (l4[0] + l4[1]) + (l4[2] + l4[3]));
         if (rescale) {
           // O may be touched now: the PV of the previous block completed before S of this
           // one (one commit tracks both), and the PV of this block waits for P_FULL below
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
+          for (int ch = 0; ch < kCols / 32; ++ch) {
             uint32_t o[32];
             tmem_ld32(tO + 32 * ch, o);
             tmem_wait_ld();
@@ -472,16 +526,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       // epilogue: O / l -> bf16 -> out[tok, head, :]
-      ok = __all_sync(0xffffffffu, wait_bounded(c, bar_addr(c, BAR_O_FULL + x), o_par,
-                                                 SITE_SOFTMAX));
+      const bool got = wait_bounded(c, bar_addr(c, BAR_O_FULL + x), o_par, SITE_SOFTMAX);
+      if constexpr (kSplit == 2) {
+        float* slot = xchg + ((xpar * 2 + x) * 2) * 128;
+        slot[half * 128 + row] = l;
+        ok = named_bar_and(2 + x, kSoftmaxThreads, got);
+        if (ok) l += slot[(half ^ 1) * 128 + row];
+        xpar ^= 1;
+      } else {
+        ok = __all_sync(0xffffffffu, got);
+      }
       if (!ok) break;
       o_par ^= 1u;
       tc_fence_after();
       const float inv_l = 1.0f / l;
       __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) +
-                           (static_cast<size_t>(tok) * 32 + head) * 128;
+                           (static_cast<size_t>(tok) * 32 + head) * 128 + kCols * half;
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
+      for (int ch = 0; ch < kCols / 32; ++ch) {
         uint32_t o[32];
         tmem_ld32(tO + 32 * ch, o);
         tmem_wait_ld();

@@ -111,7 +111,7 @@ enum : uint32_t {
 // swizzle: rows of 128 B (64 features), 8-row groups 1024 B apart (SBO); features 64..127
 // sit in the second 16 KB half of the tile.
 __device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint32_t q_tile, uint32_t k_tile) {
-#pragma unroll 1
+#pragma unroll
   for (int kk = 0; kk < 8; ++kk) {
     const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
     const uint64_t a = smem_desc_sw128(q_tile + off, 16, 1024);
@@ -125,7 +125,7 @@ __device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint32_t q_tile, uint3
 // 8-key groups 1024 B apart (SBO), the two 64-feature halves 16 KB apart (LBO).
 __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_tile,
                                          bool accumulate) {
-#pragma unroll 1
+#pragma unroll
   for (int kk = 0; kk < 8; ++kk) {
     const uint64_t b = smem_desc_sw128(v_tile + kk * 2048, kHalfBytes, 1024);
     mma_ts(tmem_o, tmem_p + kk * 8, b, kIdescPV, (accumulate || kk > 0) ? 1u : 0u);

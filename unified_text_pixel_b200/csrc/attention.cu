@@ -76,7 +76,8 @@ enum : uint32_t {
   BAR_KV_FULL = 2,                   // + slot
   BAR_KV_EMPTY = BAR_KV_FULL + kStages,
   BAR_S_FULL = BAR_KV_EMPTY + kStages,  // + tile
-  BAR_P_FULL = BAR_S_FULL + 2,
+  BAR_PA_FULL = BAR_S_FULL + 2,         // + tile: P of keys 0..63 written (O rescaled)
+  BAR_P_FULL = BAR_PA_FULL + 2,         // + tile: P of keys 64..127 written
   BAR_O_FULL = BAR_P_FULL + 2,
   BAR_O_EMPTY = BAR_O_FULL + 2,
   BAR_STALL = BAR_O_EMPTY + 2,       // debug: nothing ever arrives here
@@ -123,10 +124,11 @@ __device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint32_t q_tile, uint3
 // O_X (+)= P_X V: 8 MMAs of K = 16 keys. P (bf16, 2 per column) is read from tensor
 // memory; V is [keys, head_dim] with head_dim contiguous (N-major for the B operand):
 // 8-key groups 1024 B apart (SBO), the two 64-feature halves 16 KB apart (LBO).
+template <int kHalf>  // keys 64 * kHalf .. + 63: MMAs 4 * kHalf .. + 3
 __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_tile,
                                          bool accumulate) {
 #pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
+  for (int kk = 4 * kHalf; kk < 4 * kHalf + 4; ++kk) {
     const uint64_t b = smem_desc_sw128(v_tile + kk * 2048, kHalfBytes, 1024);
     mma_ts(tmem_o, tmem_p + kk * 8, b, kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
   }
@@ -138,18 +140,17 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint3
 #define HGX_EXP_POLY_MASK 0
 #endif
 
-// p = 2^(s * scale_log2 - mb) for the row's 128 scores, packed to bf16 pairs and stored as
-// P over the first 64 columns of S (key 2c in the low half of column c). Scale-and-shift
-// and the row sum run as paired fp32 instructions; the row sum is kept in 4 partial sums
-// (two pairs) returned in l4.
-template <bool kPoly, int N>
+// p = 2^(s * scale_log2 - mb) for scores [kFrom, kTo) of the row's N, packed to bf16 pairs
+// and stored as P over the first N/2 columns of S (key 2c in the low half of column c).
+// Scale-and-shift and the row sum run as paired fp32 instructions; the row sum is added to
+// two pair accumulators.
+template <bool kPoly, int N, int kFrom, int kTo>
 __device__ __forceinline__ void exp_store_p(const float (&s)[N], float sl2, float mb,
-                                            uint32_t tS, float (&l4)[4]) {
+                                            uint32_t tS, uint64_t (&acc)[2]) {
   const uint64_t scale2 = f2_pack(sl2, sl2);
   const uint64_t shift2 = f2_pack(-mb, -mb);
-  uint64_t acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
 #pragma unroll
-  for (int q4 = 0; q4 < N / 32; ++q4) {  // 32 keys -> 16 packed columns at a time
+  for (int q4 = kFrom / 32; q4 < kTo / 32; ++q4) {  // 32 keys -> 16 packed columns at a time
     uint32_t pk[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
@@ -167,8 +168,6 @@ __device__ __forceinline__ void exp_store_p(const float (&s)[N], float sl2, floa
     }
     tmem_st16(tS + 16 * q4, pk);
   }
-  f2_unpack(acc[0], l4[0], l4[1]);
-  f2_unpack(acc[1], l4[2], l4[3]);
 }
 
 // The CTA's items: a contiguous list from the host's assignment, or a grid-stride walk.
@@ -209,6 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(bar_addr(c, BAR_S_FULL + x), 1);
+      mbar_init(bar_addr(c, BAR_PA_FULL + x), kSoftmaxThreads);
       mbar_init(bar_addr(c, BAR_P_FULL + x), kSoftmaxThreads);
       mbar_init(bar_addr(c, BAR_O_FULL + x), 1);
       mbar_init(bar_addr(c, BAR_O_EMPTY + x), kSoftmaxThreads);
@@ -297,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ------------------------------------------------------------------ MMA issuer
       if (lane == 0) {
         uint32_t pos = 0, qf_par = 0;
-        uint32_t p_par[2] = {0, 0}, oe_par[2] = {0, 0};
+        uint32_t pa_par[2] = {0, 0}, p_par[2] = {0, 0}, oe_par[2] = {0, 0};
         bool first = true, ok = true;
         auto wait_kv = [&](uint32_t ps) {
           return wait_bounded(c, bar_addr(c, BAR_KV_FULL + ps % kStages), (ps / kStages) & 1u,
@@ -305,16 +305,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         auto slot_addr = [&](uint32_t ps) { return sRing + (ps % kStages) * kTileBytes; };
         auto release = [&](uint32_t ps) { mma_commit(bar_addr(c, BAR_KV_EMPTY + ps % kStages)); };
-        // wait until softmax X has written P (and rescaled O); before the first PV of an item
-        // also wait until the previous item's epilogue has read O
-        auto wait_p = [&](int x, bool first_pv) {
-          if (!wait_bounded(c, bar_addr(c, BAR_P_FULL + x), p_par[x], SITE_MMA)) return false;
-          p_par[x] ^= 1u;
+        // wait until softmax X has written the first half of P (and rescaled O); before the
+        // first PV of an item also wait until the previous item's epilogue has read O
+        auto wait_pa = [&](int x, bool first_pv) {
+          if (!wait_bounded(c, bar_addr(c, BAR_PA_FULL + x), pa_par[x], SITE_MMA)) return false;
+          pa_par[x] ^= 1u;
           if (first_pv && !first) {
             if (!wait_bounded(c, bar_addr(c, BAR_O_EMPTY + x), oe_par[x], SITE_MMA)) return false;
             oe_par[x] ^= 1u;
           }
           tc_fence_after();
+          return true;
+        };
+        // wait until softmax X has written the second half of P
+        auto wait_pb = [&](int x) {
+          if (!wait_bounded(c, bar_addr(c, BAR_P_FULL + x), p_par[x], SITE_MMA)) return false;
+          p_par[x] ^= 1u;
+          tc_fence_after();
+          return true;
+        };
+        // O_X (+)= P_X V in two halves of 64 keys, each issued as soon as its half of P is
+        // in tensor memory: the first half runs while the softmax exponentiates the second
+        auto pv = [&](int x, uint32_t ps, bool accumulate, bool first_pv) {
+          if (!wait_pa(x, first_pv)) return false;
+          issue_pv<0>(tmem + col_o(x), tmem + col_s(x), slot_addr(ps), accumulate);
+          if (!wait_pb(x)) return false;
+          issue_pv<1>(tmem + col_o(x), tmem + col_s(x), slot_addr(ps), accumulate);
           return true;
         };
         for (int w = first_item(p); ok && w < end_item(p); w = next_item(p, w)) {
@@ -335,12 +351,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t vpos = pos++;
             kpos = pos++;
             if (!(ok = wait_kv(vpos) && wait_kv(kpos))) break;
-            if (!(ok = wait_p(0, j == 1))) break;
-            issue_pv(tmem + col_o(0), tmem + col_s(0), slot_addr(vpos), j > 1);
+            if (!(ok = pv(0, vpos, j > 1, j == 1))) break;
             issue_qk(tmem + col_s(0), sQ, slot_addr(kpos));
             mma_commit(bar_addr(c, BAR_S_FULL + 0));
-            if (!(ok = wait_p(1, j == 1))) break;
-            issue_pv(tmem + col_o(1), tmem + col_s(1), slot_addr(vpos), j > 1);
+            if (!(ok = pv(1, vpos, j > 1, j == 1))) break;
             release(vpos);
             issue_qk(tmem + col_s(1), sQ + kTileBytes, slot_addr(kpos));
             mma_commit(bar_addr(c, BAR_S_FULL + 1));
@@ -350,11 +364,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           const uint32_t vpos = pos++;
           if (!(ok = wait_kv(vpos))) break;
-          if (!(ok = wait_p(0, n == 1))) break;
-          issue_pv(tmem + col_o(0), tmem + col_s(0), slot_addr(vpos), n > 1);
+          if (!(ok = pv(0, vpos, n > 1, n == 1))) break;
           mma_commit(bar_addr(c, BAR_O_FULL + 0));
-          if (!(ok = wait_p(1, n == 1))) break;
-          issue_pv(tmem + col_o(1), tmem + col_s(1), slot_addr(vpos), n > 1);
+          if (!(ok = pv(1, vpos, n > 1, n == 1))) break;
           mma_commit(bar_addr(c, BAR_O_FULL + 1));
           release(vpos);
           first = false;
@@ -495,15 +507,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         // key) still has m_used = -inf: exponentiate against 0, so its masked scores give
         // exact zeros and its first real maximum later rescales the all-zero O by 0
         const float mb = m_used == -INFINITY ? 0.f : m_used * sl2;
-        float l4[4];
+        // exponentials and P; the fully visible blocks may use the polynomial exp2, the
+        // others keep the MUFU instruction, which gives exact zeros for masked scores. With
+        // one warp per row, keys 0..63 come first and are published before keys 64..127 are
+        // exponentiated, so that the first half of PV overlaps the second half -- unless O
+        // must be rescaled first (rare): then both halves are published after the rescale.
+        uint64_t acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+        constexpr int kMid = kSplit == 1 ? 64 : kCols;
         if (full)
-          exp_store_p<true, kCols>(s, sl2, mb, tP, l4);   // no -inf here: polynomial allowed
+          exp_store_p<true, kCols, 0, kMid>(s, sl2, mb, tP, acc);
         else
-          exp_store_p<false, kCols>(s, sl2, mb, tP, l4);  // masked scores: MUFU gives zeros
+          exp_store_p<false, kCols, 0, kMid>(s, sl2, mb, tP, acc);
+        if (kSplit == 1 && !rescale) {
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar_addr(c, BAR_PA_FULL + x));
+        }
+        if constexpr (kMid < kCols) {
+          if (full)
+            exp_store_p<true, kCols, kMid, kCols>(s, sl2, mb, tP, acc);
+          else
+            exp_store_p<false, kCols, kMid, kCols>(s, sl2, mb, tP, acc);
+        }
+        float l4[4];
+        f2_unpack(acc[0], l4[0], l4[1]);
+        f2_unpack(acc[1], l4[2], l4[3]);
         l = fmaf(l, alpha, (l4[0] + l4[1]) + (l4[2] + l4[3]));
         if (rescale) {
           // O may be touched now: the PV of the previous block completed before S of this
-          // one (one commit tracks both), and the PV of this block waits for P_FULL below
+          // one (one commit tracks both), and the PVs of this block wait for the P barriers
+          // below
 #pragma unroll
           for (int ch = 0; ch < kCols / 32; ++ch) {
             uint32_t o[32];
@@ -522,6 +555,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_wait_st();
         tc_fence_before();
+        if (kSplit == 2 || rescale) mbar_arrive(bar_addr(c, BAR_PA_FULL + x));
         mbar_arrive(bar_addr(c, BAR_P_FULL + x));
       }
       if (!ok) break;

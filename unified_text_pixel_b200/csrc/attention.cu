@@ -31,6 +31,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "exp2_poly.h"
 #include "kernels.h"
@@ -64,6 +65,13 @@ constexpr uint32_t kRegsHigh = kSplit == 1 ? 192 : 104;  // softmax warpgroups
 #define HGX_KV_STAGES 4
 #endif
 constexpr int kStages = HGX_KV_STAGES;        // K/V ring slots
+#ifndef HGX_P_PARTS
+#define HGX_P_PARTS 2
+#endif
+// P of a tile is published in this many parts of 128 / kPParts keys (one warp per row), so
+// that the PV MMAs of the first parts overlap the exponentials of the later ones
+constexpr int kPParts = HGX_P_PARTS;
+static_assert(kPParts == 1 || kPParts == 2 || kPParts == 4, "P parts");
 constexpr uint32_t kTileBytes = 32768;        // 128 rows x 128 bf16
 constexpr uint32_t kHalfBytes = 16384;        // 128 rows x 64 bf16 (one 128-byte swizzle span)
 constexpr uint32_t kQBytes = 2 * kTileBytes;  // both Q tiles of an item
@@ -76,8 +84,8 @@ enum : uint32_t {
   BAR_KV_FULL = 2,                   // + slot
   BAR_KV_EMPTY = BAR_KV_FULL + kStages,
   BAR_S_FULL = BAR_KV_EMPTY + kStages,  // + tile
-  BAR_PA_FULL = BAR_S_FULL + 2,         // + tile: P of keys 0..63 written (O rescaled)
-  BAR_P_FULL = BAR_PA_FULL + 2,         // + tile: P of keys 64..127 written
+  BAR_PA_FULL = BAR_S_FULL + 2,         // + tile * (kPParts - 1) + part: that part of P written
+  BAR_P_FULL = BAR_PA_FULL + 2 * (kPParts - 1),  // + tile: the last part of P written
   BAR_O_FULL = BAR_P_FULL + 2,
   BAR_O_EMPTY = BAR_O_FULL + 2,
   BAR_STALL = BAR_O_EMPTY + 2,       // debug: nothing ever arrives here
@@ -124,11 +132,11 @@ __device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint32_t q_tile, uint3
 // O_X (+)= P_X V: 8 MMAs of K = 16 keys. P (bf16, 2 per column) is read from tensor
 // memory; V is [keys, head_dim] with head_dim contiguous (N-major for the B operand):
 // 8-key groups 1024 B apart (SBO), the two 64-feature halves 16 KB apart (LBO).
-template <int kHalf>  // keys 64 * kHalf .. + 63: MMAs 4 * kHalf .. + 3
+template <int kFrom, int kTo>  // MMAs kFrom .. kTo - 1: keys 16 * kFrom .. 16 * kTo - 1
 __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_tile,
                                          bool accumulate) {
 #pragma unroll
-  for (int kk = 4 * kHalf; kk < 4 * kHalf + 4; ++kk) {
+  for (int kk = kFrom; kk < kTo; ++kk) {
     const uint64_t b = smem_desc_sw128(v_tile + kk * 2048, kHalfBytes, 1024);
     mma_ts(tmem_o, tmem_p + kk * 8, b, kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
   }
@@ -139,6 +147,7 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint3
 // ex2 (fully visible blocks only). 0 = never.
 #define HGX_EXP_POLY_MASK 0
 #endif
+constexpr bool kExpPolyOn = HGX_EXP_POLY_MASK != 0;
 
 // p = 2^(s * scale_log2 - mb) for scores [kFrom, kTo) of the row's N, packed to bf16 pairs
 // and stored as P over the first N/2 columns of S (key 2c in the low half of column c).
@@ -208,7 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(bar_addr(c, BAR_S_FULL + x), 1);
-      mbar_init(bar_addr(c, BAR_PA_FULL + x), kSoftmaxThreads);
+      for (int i = 0; i < kPParts - 1; ++i)
+        mbar_init(bar_addr(c, BAR_PA_FULL + x * (kPParts - 1) + i), kSoftmaxThreads);
       mbar_init(bar_addr(c, BAR_P_FULL + x), kSoftmaxThreads);
       mbar_init(bar_addr(c, BAR_O_FULL + x), 1);
       mbar_init(bar_addr(c, BAR_O_EMPTY + x), kSoftmaxThreads);
@@ -297,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ------------------------------------------------------------------ MMA issuer
       if (lane == 0) {
         uint32_t pos = 0, qf_par = 0;
-        uint32_t pa_par[2] = {0, 0}, p_par[2] = {0, 0}, oe_par[2] = {0, 0};
+        uint32_t pa_par[2] = {0, 0}, p_par[2] = {0, 0}, oe_par[2] = {0, 0};  // pa: all parts share it
         bool first = true, ok = true;
         auto wait_kv = [&](uint32_t ps) {
           return wait_bounded(c, bar_addr(c, BAR_KV_FULL + ps % kStages), (ps / kStages) & 1u,
@@ -305,32 +315,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         auto slot_addr = [&](uint32_t ps) { return sRing + (ps % kStages) * kTileBytes; };
         auto release = [&](uint32_t ps) { mma_commit(bar_addr(c, BAR_KV_EMPTY + ps % kStages)); };
-        // wait until softmax X has written the first half of P (and rescaled O); before the
-        // first PV of an item also wait until the previous item's epilogue has read O
-        auto wait_pa = [&](int x, bool first_pv) {
-          if (!wait_bounded(c, bar_addr(c, BAR_PA_FULL + x), pa_par[x], SITE_MMA)) return false;
-          pa_par[x] ^= 1u;
-          if (first_pv && !first) {
+        // wait until softmax X has written part `part` of P (the first part: and rescaled O);
+        // before the first PV of an item also wait until the previous item's epilogue has
+        // read O. The parts other than the last have barriers of their own, which all
+        // complete once per block, so they share one parity.
+        auto wait_part = [&](int x, int part, bool first_pv) {
+          const bool last = part == kPParts - 1;
+          const uint32_t bar = last ? BAR_P_FULL + x : BAR_PA_FULL + x * (kPParts - 1) + part;
+          if (!wait_bounded(c, bar_addr(c, bar), last ? p_par[x] : pa_par[x], SITE_MMA)) return false;
+          if (last) p_par[x] ^= 1u;
+          else if (part == kPParts - 2) pa_par[x] ^= 1u;
+          if (part == 0 && first_pv && !first) {
             if (!wait_bounded(c, bar_addr(c, BAR_O_EMPTY + x), oe_par[x], SITE_MMA)) return false;
             oe_par[x] ^= 1u;
           }
           tc_fence_after();
           return true;
         };
-        // wait until softmax X has written the second half of P
-        auto wait_pb = [&](int x) {
-          if (!wait_bounded(c, bar_addr(c, BAR_P_FULL + x), p_par[x], SITE_MMA)) return false;
-          p_par[x] ^= 1u;
-          tc_fence_after();
-          return true;
-        };
-        // O_X (+)= P_X V in two halves of 64 keys, each issued as soon as its half of P is
-        // in tensor memory: the first half runs while the softmax exponentiates the second
+        // O_X (+)= P_X V in kPParts parts, each issued as soon as its part of P is in tensor
+        // memory: the first parts run while the softmax exponentiates the later ones
         auto pv = [&](int x, uint32_t ps, bool accumulate, bool first_pv) {
-          if (!wait_pa(x, first_pv)) return false;
-          issue_pv<0>(tmem + col_o(x), tmem + col_s(x), slot_addr(ps), accumulate);
-          if (!wait_pb(x)) return false;
-          issue_pv<1>(tmem + col_o(x), tmem + col_s(x), slot_addr(ps), accumulate);
+          constexpr int kStep = 8 / kPParts;
+          if (!wait_part(x, 0, first_pv)) return false;
+          issue_pv<0, kStep>(tmem + col_o(x), tmem + col_s(x), slot_addr(ps), accumulate);
+          if constexpr (kPParts >= 2) {
+            if (!wait_part(x, 1, first_pv)) return false;
+            issue_pv<kStep, 2 * kStep>(tmem + col_o(x), tmem + col_s(x), slot_addr(ps), accumulate);
+          }
+          if constexpr (kPParts == 4) {
+            if (!wait_part(x, 2, first_pv)) return false;
+            issue_pv<2 * kStep, 3 * kStep>(tmem + col_o(x), tmem + col_s(x), slot_addr(ps), accumulate);
+            if (!wait_part(x, 3, first_pv)) return false;
+            issue_pv<3 * kStep, 4 * kStep>(tmem + col_o(x), tmem + col_s(x), slot_addr(ps), accumulate);
+          }
           return true;
         };
         for (int w = first_item(p); ok && w < end_item(p); w = next_item(p, w)) {
@@ -507,27 +524,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         // key) still has m_used = -inf: exponentiate against 0, so its masked scores give
         // exact zeros and its first real maximum later rescales the all-zero O by 0
         const float mb = m_used == -INFINITY ? 0.f : m_used * sl2;
-        // exponentials and P; the fully visible blocks may use the polynomial exp2, the
-        // others keep the MUFU instruction, which gives exact zeros for masked scores. With
-        // one warp per row, keys 0..63 come first and are published before keys 64..127 are
-        // exponentiated, so that the first half of PV overlaps the second half -- unless O
-        // must be rescaled first (rare): then both halves are published after the rescale.
+        // exponentials and P. With one warp per row, P is written in kPParts parts and each
+        // part but the last is published before the next is exponentiated, so that the PV
+        // MMAs of the early parts overlap the later exponentials -- unless O must be rescaled
+        // first (rare): then every part is published after the rescale.
         uint64_t acc[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
-        constexpr int kMid = kSplit == 1 ? 64 : kCols;
-        if (full)
-          exp_store_p<true, kCols, 0, kMid>(s, sl2, mb, tP, acc);
-        else
-          exp_store_p<false, kCols, 0, kMid>(s, sl2, mb, tP, acc);
-        if (kSplit == 1 && !rescale) {
+        constexpr int kParts = kSplit == 1 ? kPParts : 1;
+        constexpr int kW = kCols / kParts;  // keys per part
+        const bool early = kParts > 1 && !rescale;
+        auto publish = [&](int part) {
           tmem_wait_st();
           tc_fence_before();
-          mbar_arrive(bar_addr(c, BAR_PA_FULL + x));
-        }
-        if constexpr (kMid < kCols) {
-          if (full)
-            exp_store_p<true, kCols, kMid, kCols>(s, sl2, mb, tP, acc);
+          mbar_arrive(bar_addr(c, BAR_PA_FULL + x * (kPParts - 1) + part));
+        };
+        auto exp_part = [&](auto from_c, auto to_c) {
+          constexpr int kFrom = decltype(from_c)::value, kTo = decltype(to_c)::value;
+          if (kExpPolyOn && full)
+            exp_store_p<true, kCols, kFrom, kTo>(s, sl2, mb, tP, acc);  // no -inf: polynomial allowed
           else
-            exp_store_p<false, kCols, kMid, kCols>(s, sl2, mb, tP, acc);
+            exp_store_p<false, kCols, kFrom, kTo>(s, sl2, mb, tP, acc);  // MUFU: zeros for -inf
+        };
+        exp_part(std::integral_constant<int, 0>{}, std::integral_constant<int, kW>{});
+        if constexpr (kParts >= 2) {
+          if (early) publish(0);
+          exp_part(std::integral_constant<int, kW>{}, std::integral_constant<int, 2 * kW>{});
+        }
+        if constexpr (kParts == 4) {
+          if (early) publish(1);
+          exp_part(std::integral_constant<int, 2 * kW>{}, std::integral_constant<int, 3 * kW>{});
+          if (early) publish(2);
+          exp_part(std::integral_constant<int, 3 * kW>{}, std::integral_constant<int, 4 * kW>{});
         }
         float l4[4];
         f2_unpack(acc[0], l4[0], l4[1]);
@@ -555,7 +581,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        if (kSplit == 2 || rescale) mbar_arrive(bar_addr(c, BAR_PA_FULL + x));
+        if (!early)  // every part at once
+          for (int i = 0; i < kPParts - 1; ++i) mbar_arrive(bar_addr(c, BAR_PA_FULL + x * (kPParts - 1) + i));
         mbar_arrive(bar_addr(c, BAR_P_FULL + x));
       }
       if (!ok) break;

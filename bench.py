@@ -373,7 +373,9 @@ def run_gpu(args):
             out_h.copy_(outs[b], non_blocking=True)
             down_done[b].record(s_down)
 
-    e2e_steps = max(3, min(args.steps, 20))
+    e2e_steps = max(3, args.steps)  # as many steps as the device-timed region: the fill and drain
+    # of the copy pipeline (one upload before the first forward, one forward and download
+    # after the last upload) are then a small part of the timed region
     for i in range(3):
         e2e_step(i)
     torch.cuda.synchronize()

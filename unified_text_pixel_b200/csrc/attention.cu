@@ -24,6 +24,10 @@
 // tensor memory. The MMA warp interleaves the tiles so that one tile's softmax runs while
 // the tensor core works on the other's QK^T and PV:
 //   S0(0) S1(0) | PV0(j-1) S0(j) PV1(j-1) S1(j) | ... | PV0(n-1) PV1(n-1)
+// A softmax warp publishes P in two halves (keys 0..63, then 64..127), and the MMA warp
+// issues the PV MMAs of the first half while the second half is being exponentiated: a
+// key block's period is set by each tile's chain S -> softmax -> P -> PV -> S, so work
+// moved off that chain is time saved.
 // Online softmax keeps the running maximum that was last used for exponentiation and only
 // rescales O (in tensor memory) and the row sum when the maximum grows by more than 2^8,
 // so probabilities stay below 256 and O is rarely touched.
@@ -51,8 +55,9 @@ using namespace waits;
 // Softmax warps per row of a tile: 1 -- one thread holds a whole 128-column row; 2 -- two
 // warps on the same tensor-memory lanes each take 64 columns (twice the softmax warps,
 // half the dependent work per warp; the row maximum is exchanged through shared memory).
-// Both give the same results within rounding; on B200 split 2 measured no faster (within
-// 1% at 8k-16k tokens, 5% slower at 1k), so 1 is the default.
+// Both give the same results within rounding; on B200 split 2 measured no faster (the
+// exponentials of a row stay on the same SM sub-partition, whose MUFU and issue slots
+// they share), so 1 is the default.
 constexpr int kSplit = HGX_SOFTMAX_SPLIT;
 static_assert(kSplit == 1 || kSplit == 2, "softmax split");
 constexpr int kCols = 128 / kSplit;               // score columns per softmax thread

@@ -194,6 +194,17 @@ def cpu_oracle_sample(w, budget_s=15.0, seed=0):
     return flops / elapsed / 1e12, rows_done, elapsed, threads
 
 
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def _blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -230,7 +241,7 @@ def run_reference(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": _config_dict(w, None),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
-                         "sample": sample},
+                         "cpu": _cpu_model(), "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -437,6 +448,8 @@ def run_gpu(args):
                 "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps,
                 "how": "hgx_attn_forward per step; uploads and downloads on their own streams, "
                        "overlapping neighbouring steps' forwards"},
+        "exp_offload": "none: MUFU ex2.approx for every score (a polynomial exp2 on the FMA pipe "
+                       "for part of the scores measured slower on B200)",
         "gpu_launches": (1 + (sum(1 for b in range(len(w.batches)) if first_rows[b] < w.lengths[b])
                               if first_rows else 1)) * args.steps,
         "clocks": clk.summary(),
@@ -446,6 +459,7 @@ def run_gpu(args):
         _log("cpu baseline (oracle)")
         v, rows, secs, threads = cpu_oracle_sample(w, budget_s=args.cpu_seconds)
         line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                                "cpu": _cpu_model(),
                                 "sample": f"{rows} random rows of {w.name} (all 32 query heads, fp64) in {secs:.1f} s"}
     a.close()
     if dist:

@@ -123,28 +123,29 @@ enum : uint32_t {
 
 // S_X = Q_X K^T over head_dim 128: 8 MMAs of K = 16. Both operands K-major with 128-byte
 // swizzle: rows of 128 B (64 features), 8-row groups 1024 B apart (SBO); features 64..127
-// sit in the second 16 KB half of the tile.
-__device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint32_t q_tile, uint32_t k_tile) {
+// sit in the second 16 KB half of the tile. The tiles' descriptors are passed in: MMA k
+// reads (k >> 2) * 16 KB + (k & 3) * 32 B further on, which adds that offset >> 4 to the
+// descriptor's 14-bit start-address field (shared addresses stay below 256 KB, so the
+// field never carries into the next one).
+__device__ __forceinline__ void issue_qk(uint32_t tmem_s, uint64_t q_desc, uint64_t k_desc) {
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk) {
-    const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-    const uint64_t a = smem_desc_sw128(q_tile + off, 16, 1024);
-    const uint64_t b = smem_desc_sw128(k_tile + off, 16, 1024);
-    mma_ss(tmem_s, a, b, kIdescQK, kk > 0 ? 1u : 0u);
+    const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+    mma_ss(tmem_s, q_desc + off, k_desc + off, kIdescQK, kk > 0 ? 1u : 0u);
   }
 }
 
 // O_X (+)= P_X V: 8 MMAs of K = 16 keys. P (bf16, 2 per column) is read from tensor
 // memory; V is [keys, head_dim] with head_dim contiguous (N-major for the B operand):
 // 8-key groups 1024 B apart (SBO), the two 64-feature halves 16 KB apart (LBO).
+// MMA k reads keys 16k.. of V, 2 KB further on (descriptor passed in, as for issue_qk).
 template <int kFrom, int kTo>  // MMAs kFrom .. kTo - 1: keys 16 * kFrom .. 16 * kTo - 1
-__device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_tile,
+__device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint64_t v_desc,
                                          bool accumulate) {
 #pragma unroll
-  for (int kk = kFrom; kk < kTo; ++kk) {
-    const uint64_t b = smem_desc_sw128(v_tile + kk * 2048, kHalfBytes, 1024);
-    mma_ts(tmem_o, tmem_p + kk * 8, b, kIdescPV, (accumulate || kk > 0) ? 1u : 0u);
-  }
+  for (int kk = kFrom; kk < kTo; ++kk)
+    mma_ts(tmem_o, tmem_p + kk * 8, v_desc + kk * (2048 >> 4), kIdescPV,
+           (accumulate || kk > 0) ? 1u : 0u);
 }
 
 #ifndef HGX_EXP_POLY_MASK
@@ -318,7 +319,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           return wait_bounded(c, bar_addr(c, BAR_KV_FULL + ps % kStages), (ps / kStages) & 1u,
                               SITE_MMA);
         };
-        auto slot_addr = [&](uint32_t ps) { return sRing + (ps % kStages) * kTileBytes; };
+        // descriptors of both Q tiles and of K / V in ring slot 0 (slot s: + s * 32 KB >> 4)
+        const uint64_t dq0 = smem_desc_sw128(sQ, 16, 1024);
+        const uint64_t dq1 = smem_desc_sw128(sQ + kTileBytes, 16, 1024);
+        const uint64_t dk0 = smem_desc_sw128(sRing, 16, 1024);
+        const uint64_t dv0 = smem_desc_sw128(sRing, kHalfBytes, 1024);
+        auto kdesc = [&](uint32_t ps) { return dk0 + (ps % kStages) * (kTileBytes >> 4); };
+        auto vdesc = [&](uint32_t ps) { return dv0 + (ps % kStages) * (kTileBytes >> 4); };
         auto release = [&](uint32_t ps) { mma_commit(bar_addr(c, BAR_KV_EMPTY + ps % kStages)); };
         // wait until softmax X has written part `part` of P (the first part: and rescaled O);
         // before the first PV of an item also wait until the previous item's epilogue has
@@ -342,16 +349,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto pv = [&](int x, uint32_t ps, bool accumulate, bool first_pv) {
           constexpr int kStep = 8 / kPParts;
           if (!wait_part(x, 0, first_pv)) return false;
-          issue_pv<0, kStep>(tmem + col_o(x), tmem + col_s(x), slot_addr(ps), accumulate);
+          issue_pv<0, kStep>(tmem + col_o(x), tmem + col_s(x), vdesc(ps), accumulate);
           if constexpr (kPParts >= 2) {
             if (!wait_part(x, 1, first_pv)) return false;
-            issue_pv<kStep, 2 * kStep>(tmem + col_o(x), tmem + col_s(x), slot_addr(ps), accumulate);
+            issue_pv<kStep, 2 * kStep>(tmem + col_o(x), tmem + col_s(x), vdesc(ps), accumulate);
           }
           if constexpr (kPParts == 4) {
             if (!wait_part(x, 2, first_pv)) return false;
-            issue_pv<2 * kStep, 3 * kStep>(tmem + col_o(x), tmem + col_s(x), slot_addr(ps), accumulate);
+            issue_pv<2 * kStep, 3 * kStep>(tmem + col_o(x), tmem + col_s(x), vdesc(ps), accumulate);
             if (!wait_part(x, 3, first_pv)) return false;
-            issue_pv<3 * kStep, 4 * kStep>(tmem + col_o(x), tmem + col_s(x), slot_addr(ps), accumulate);
+            issue_pv<3 * kStep, 4 * kStep>(tmem + col_o(x), tmem + col_s(x), vdesc(ps), accumulate);
           }
           return true;
         };
@@ -363,9 +370,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t kpos = pos++;
           if (!(ok = wait_kv(kpos))) break;
           tc_fence_after();
-          issue_qk(tmem + col_s(0), sQ, slot_addr(kpos));
+          issue_qk(tmem + col_s(0), dq0, kdesc(kpos));
           mma_commit(bar_addr(c, BAR_S_FULL + 0));
-          issue_qk(tmem + col_s(1), sQ + kTileBytes, slot_addr(kpos));
+          issue_qk(tmem + col_s(1), dq1, kdesc(kpos));
           mma_commit(bar_addr(c, BAR_S_FULL + 1));
           if (n == 1) mma_commit(bar_addr(c, BAR_Q_EMPTY));
           release(kpos);
@@ -374,11 +381,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             kpos = pos++;
             if (!(ok = wait_kv(vpos) && wait_kv(kpos))) break;
             if (!(ok = pv(0, vpos, j > 1, j == 1))) break;
-            issue_qk(tmem + col_s(0), sQ, slot_addr(kpos));
+            issue_qk(tmem + col_s(0), dq0, kdesc(kpos));
             mma_commit(bar_addr(c, BAR_S_FULL + 0));
             if (!(ok = pv(1, vpos, j > 1, j == 1))) break;
             release(vpos);
-            issue_qk(tmem + col_s(1), sQ + kTileBytes, slot_addr(kpos));
+            issue_qk(tmem + col_s(1), dq1, kdesc(kpos));
             mma_commit(bar_addr(c, BAR_S_FULL + 1));
             if (j == n - 1) mma_commit(bar_addr(c, BAR_Q_EMPTY));
             release(kpos);

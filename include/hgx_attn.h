@@ -209,6 +209,9 @@ hgx_status hgx_attn_sync_status(hgx_attn_handle* h, void* stream);
 #define HGX_DEBUG_CHECKED 1u    /* every device call ends with hgx_attn_sync_status */
 #define HGX_DEBUG_STALL_TEST 2u /* attention: one softmax warpgroup first waits on a barrier
                                    that nothing arrives at, so its bounded wait runs out */
+#define HGX_DEBUG_FAIL_ALLOC 4u /* the next device allocation of the planner scratch reports
+                                   HGX_ERR_OOM instead of allocating (one-shot: the flag
+                                   clears itself); nothing is launched by that call */
 
 /* Sets debug flags and the bound of every device wait in nanoseconds (0 keeps the
  * default of 2 s). The HGX_DEBUG environment variable (an integer) sets the initial

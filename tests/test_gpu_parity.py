@@ -343,6 +343,31 @@ def test_empty_batch_is_a_no_op(hgx):
     a.forward(z, z, z, z, z, z, z, [0, 0], np.zeros((0, 3)), [0, 0])
 
 
+def test_injected_allocation_failure_reports_oom_and_handle_recovers(hgx):
+    """A one-shot test hook makes the planner's scratch allocation fail: the forward returns
+    HGX_ERR_OOM before launching anything (q and k stay untouched), and the next call on the
+    same handle allocates and matches the oracle."""
+    H, _ = hgx
+    w = W.config(0)
+    t, d = _device_inputs(w)
+    a = H.Attention()  # a fresh handle: its first forward has to allocate
+    try:
+        out = torch.empty_like(d["q"])
+        q0, k0 = d["q"].clone(), d["k"].clone()
+        a.set_debug(H.HGX_DEBUG_FAIL_ALLOC, 0)
+        with pytest.raises(H.HgxError) as e:
+            a.forward(d["q"], d["k"], d["v"], out, d["pos"], d["wq"], d["wk"], *_desc(w))
+        assert e.value.status == H.HGX_ERR_OOM
+        assert "injected" in a.last_error()
+        torch.cuda.synchronize()
+        assert torch.equal(d["q"], q0) and torch.equal(d["k"], k0)
+        a.forward(d["q"], d["k"], d["v"], out, d["pos"], d["wq"], d["wk"], *_desc(w))
+        ref, _, _ = _oracle_full(w, t)
+        _compare(out.float().cpu().numpy(), ref, "after-injected-oom")
+    finally:
+        a.close()
+
+
 def test_bounded_wait_reports_timeout_and_context_survives(hgx):
     """A softmax warpgroup waits on a barrier that nothing arrives at; its bounded wait
     runs out, the kernel drains and exits, the host sees HGX_ERR_TIMEOUT, and the next

@@ -226,6 +226,9 @@ def test_set_debug_rejects_unknown_flags():
     with pytest.raises(B.HgxError):
         a.set_debug(0x80)
     a.set_debug(B.HGX_DEBUG_CHECKED, 10_000_000)
+    a.set_debug(B.HGX_DEBUG_FAIL_ALLOC | B.HGX_DEBUG_CHECKED | B.HGX_DEBUG_STALL_TEST)
+    with pytest.raises(B.HgxError):
+        a.set_debug(8)
     a.close()
 
 

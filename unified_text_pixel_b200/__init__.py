@@ -20,6 +20,7 @@ from .binding import (  # noqa: F401
     HGX_TILE_FULL,
     HGX_DEBUG_CHECKED,
     HGX_DEBUG_STALL_TEST,
+    HGX_DEBUG_FAIL_ALLOC,
     HGX_ROPE_MROPE_INTERLEAVED,
     HGX_ROPE_2D_ALTERNATING,
     HGX_ROPE_2D_HALVES,

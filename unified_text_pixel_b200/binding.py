@@ -15,7 +15,7 @@ import numpy as np
 HGX_OK, HGX_ERR_INVALID_ARG, HGX_ERR_UNSUPPORTED, HGX_ERR_OOM, HGX_ERR_CUDA, HGX_ERR_TIMEOUT = range(6)
 HGX_SEG_CAUSAL, HGX_SEG_FULL_SEQUENCE, HGX_SEG_FULL_IN_SEGMENT, HGX_SEG_GEN_IMAGE = 0, 1, 2, 3
 HGX_TILE_SKIP, HGX_TILE_PARTIAL, HGX_TILE_FULL = 0, 1, 2
-HGX_DEBUG_CHECKED, HGX_DEBUG_STALL_TEST = 1, 2
+HGX_DEBUG_CHECKED, HGX_DEBUG_STALL_TEST, HGX_DEBUG_FAIL_ALLOC = 1, 2, 4
 HGX_ROPE_MROPE_INTERLEAVED, HGX_ROPE_2D_ALTERNATING, HGX_ROPE_2D_HALVES = 0, 1, 2
 
 _STATUS = {0: "HGX_OK", 1: "HGX_ERR_INVALID_ARG", 2: "HGX_ERR_UNSUPPORTED", 3: "HGX_ERR_OOM",

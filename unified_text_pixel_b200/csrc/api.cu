@@ -208,6 +208,10 @@ hgx_status prepare_plan(hgx_attn_handle* h, cudaStream_t stream, int32_t batch,
   size_t need = 0;
   for (const Upload& u : up) {
     if (u.bytes > *u.cap) {
+      if (h->flags & HGX_DEBUG_FAIL_ALLOC) {  // injected failure (test hook), one-shot
+        h->flags &= ~HGX_DEBUG_FAIL_ALLOC;
+        return fail(h, HGX_ERR_OOM, "cudaMalloc of the planner scratch failed (injected)");
+      }
       if (*u.dst) cudaFree(*u.dst);
       *u.dst = nullptr;
       *u.cap = 0;
@@ -649,7 +653,7 @@ hgx_status hgx_attn_sync_status(hgx_attn_handle* h, void* stream) {
 
 hgx_status hgx_attn_set_debug(hgx_attn_handle* h, uint32_t flags, uint64_t wait_limit_ns) {
   if (!h) return HGX_ERR_INVALID_ARG;
-  if (flags & ~(HGX_DEBUG_CHECKED | HGX_DEBUG_STALL_TEST))
+  if (flags & ~(HGX_DEBUG_CHECKED | HGX_DEBUG_STALL_TEST | HGX_DEBUG_FAIL_ALLOC))
     return fail(h, HGX_ERR_INVALID_ARG, "unknown debug flag");
   h->flags = flags;
   h->wait_limit_ns = wait_limit_ns ? wait_limit_ns : 2000000000ull;

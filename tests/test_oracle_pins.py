@@ -324,3 +324,39 @@ def test_layer_rows_agrees_with_layer_forward():
     y_r, att_r = O.layer_rows(lt["x"], lt["w_qkv"], lt["w_o"], pos, lt["wq"], lt["wk"], cu, segs, cu_segs, rows)
     np.testing.assert_allclose(att_r, att[rows], rtol=0, atol=1e-12)
     np.testing.assert_allclose(y_r, y[rows], rtol=0, atol=1e-11)
+
+
+@pytest.mark.parametrize("case", ["random_holes", "random_multi", "random_empty", "params"])
+def test_attention_rows_agrees_with_forward(case):
+    """The sampled-rows oracle that the full-size GPU tests and the CPU baseline use equals
+    the whole-sequence oracle (itself pinned to library SDPA and 50-digit brute force) on
+    EVERY row of small packed batches: several batch elements (so a row must take the keys
+    of its own element), empty elements, all four segment kinds including Gen Image holes,
+    and non-default theta / eps / scale (so each is passed through). A wrong head mapping
+    (h % Hkv), a dropped scale, a prologue over the wrong key range or a mask row of the
+    wrong token each fails here."""
+    if case == "random_holes":
+        w = W.random_workload(71, max_batch=3, max_len=160, kinds=(0, 1, 2, 3, 3))
+        kw = {}
+    elif case == "random_multi":
+        w = W.random_workload(72, max_batch=4, max_len=150)
+        kw = {}
+    elif case == "random_empty":
+        w = W.custom("with_empty", [[(13, W.CAUSAL), (20, W.FULL_SEQUENCE)], [], [(7, W.FULL_IN_SEGMENT), (9, W.CAUSAL)]],
+                     seed=73)
+        kw = {}
+    else:
+        w = W.custom("params", [[(11, W.CAUSAL), (17, W.GEN_IMAGE), (6, W.CAUSAL)], [(21, W.FULL_SEQUENCE)]], seed=74)
+        kw = dict(theta=1.0e4, eps=0.25, scale=0.05)
+    t = W.tensors(w)
+    segs, cu_segs = W.flat_segments(w)
+    pos, cu = W.positions(w), W.cu_seqlens(w)
+    assert len(cu) - 1 >= 2 or case == "random_holes"
+    ref, _, _ = O.forward(t["q"], t["k"], t["v"], pos, t["wq"], t["wk"], cu, segs, cu_segs, **kw)
+    rows = list(range(w.total_tokens))
+    got = O.attention_rows(t["q"], t["k"], t["v"], pos, t["wq"], t["wk"], cu, segs, cu_segs, rows, **kw)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+    # an unordered subset with a repeat gives the same rows
+    sub = [rows[-1], rows[0], rows[len(rows) // 2], rows[0]]
+    got_sub = O.attention_rows(t["q"], t["k"], t["v"], pos, t["wq"], t["wk"], cu, segs, cu_segs, sub, **kw)
+    np.testing.assert_allclose(got_sub, ref[sub], rtol=0, atol=1e-12)

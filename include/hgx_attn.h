@@ -41,8 +41,11 @@
  *   pos  int32 [T, 3]  (t, h, w) position of each token -- read only
  *   wq, wk bf16 [128]  RMSNorm weights                  -- read only
  * Every device pointer must be non-null (when T > 0) and 16-byte aligned; out must not
- * overlap q, k or v. V must be finite: the kernel multiplies masked probabilities (exact
- * zeros) with key rows of the neighbouring batch element, and 0 * inf is NaN.
+ * overlap q, k or v. V must be finite within each batch element: a row's masked
+ * probabilities (exact zeros) meet V rows of its own element that it cannot see, and
+ * 0 * inf is NaN. V rows of other batch elements never reach a row's output: where a
+ * 128-key block runs past the end of an element, the kernel zeroes the next element's V
+ * rows in shared memory before the P V product.
  *
  * Segments: for batch element b, segs[cu_segs[b] .. cu_segs[b+1]) describe its tokens in
  * order. Each has a start local to the element, a length >= 1 and a kind. They must tile
@@ -175,6 +178,44 @@ hgx_status hgx_attn_attention(hgx_attn_handle* h, void* stream, const void* q, c
                               const int32_t* cu_seqlens_host, const hgx_segment* segs_host,
                               const int32_t* cu_segs_host);
 
+/* ---------------------------------------------------------------------------------------
+ * The attention layer around the core: the QKV projection in front of it and the output
+ * projection behind it. Sizes from "hidream-o1-p100a" model card, "What this model is":
+ * hidden size 4096, 32 query heads over 8 KV heads at head_dim 128, so the projection
+ * maps 4096 features to 32*128 + 2*8*128 = 6144 and the output projection 4096 -> 4096.
+ * Weights are row-major [out, in] bf16 (y = x W^T):
+ *   w_qkv  bf16 [6144, 4096]: rows 0..4095 the 32 query heads (128 rows each, head h at
+ *          rows 128h..128h+127), rows 4096..5119 the 8 key heads, rows 5120..6143 the 8
+ *          value heads
+ *   w_o    bf16 [4096, 4096]: column 128h + d reads feature d of query head h
+ *   x      bf16 [T, 4096] hidden states; attn bf16 [T, 32, 128]; y bf16 [T, 4096]
+ * All pointers device, non-null and 16-byte aligned; T = total_tokens <= 2^19 - 1. The
+ * GEMMs run on the tensor cores with fp32 accumulation and round to bf16. */
+
+/* q' = rope(rmsnorm(x Wq^T) * wq), k' = rope(rmsnorm(x Wk^T) * wk), v = x Wv^T: the
+ * projection with the prologue's RMSNorm and rotation fused into its epilogue (no q/k
+ * round trip through memory). q [T,32,128], k and v [T,8,128] are written; positions and
+ * norm weights as in hgx_attn_forward. Errors: INVALID_ARG (pointer, size), CUDA, OOM
+ * (the per-call (cos, sin) table of the rotation is allocated by the handle). */
+hgx_status hgx_attn_qkv_projection(hgx_attn_handle* h, void* stream, const void* x,
+                                   const void* w_qkv, void* q, void* k, void* v,
+                                   const int32_t* pos_thw, const void* q_norm_w,
+                                   const void* k_norm_w, int32_t total_tokens);
+
+/* y = attn W_o^T, attn read as [T, 4096]. Errors: INVALID_ARG (pointer, size), CUDA. */
+hgx_status hgx_attn_out_projection(hgx_attn_handle* h, void* stream, const void* attn,
+                                   const void* w_o, void* y, int32_t total_tokens);
+
+/* The whole layer: hgx_attn_qkv_projection into q, k, v, masked attention into attn
+ * (segment descriptor as in hgx_attn_forward), hgx_attn_out_projection into y. q, k, v
+ * and attn are caller-provided intermediates; attn must not overlap q, k or v. */
+hgx_status hgx_attn_layer_forward(hgx_attn_handle* h, void* stream, const void* x,
+                                  const void* w_qkv, const void* w_o, void* q, void* k, void* v,
+                                  void* attn, void* y, const int32_t* pos_thw,
+                                  const void* q_norm_w, const void* k_norm_w, int32_t batch,
+                                  const int32_t* cu_seqlens_host, const hgx_segment* segs_host,
+                                  const int32_t* cu_segs_host);
+
 /* Host only (no GPU needed). Exclusive key limit lim(i) of every packed row, local to its
  * batch element: row i sees keys [0, lim(i)) minus the keys of gen_image segments before
  * its own segment. lim_out has room for cap entries; T entries are written. Errors:
@@ -225,21 +266,28 @@ hgx_status hgx_attn_set_debug(hgx_attn_handle* h, uint32_t flags, uint64_t wait_
  * process whose device footprint must not grow after start-up. It needs no handle (creating
  * one allocates) and calls no cudaMalloc, cudaFree, cudaMallocHost or heap allocation.
  *
- * Scratch (per-row key limits, work list, error word) lives in one fixed-size device array
- * inside the library (about 145 KB, held by every GPU that loads the library until the
- * process exits); planning uses fixed-size static host buffers. Hence the limits:
- * at most HGX_NOALLOC_MAX_TOKENS packed tokens and HGX_NOALLOC_MAX_BATCH batch elements,
- * and no gen_image segments; other requests return HGX_ERR_UNSUPPORTED before any device
- * work.
+ * Scratch (per-row key limits, work list, per-CTA item offsets, error word) lives in one
+ * fixed-size device array inside the library (about 145 KB, held by every GPU that loads
+ * the library until the process exits); planning uses fixed-size static host buffers. Hence
+ * the limits: at most HGX_NOALLOC_MAX_TOKENS packed tokens and HGX_NOALLOC_MAX_BATCH batch
+ * elements, and no gen_image segments; other requests return HGX_ERR_UNSUPPORTED before
+ * any device work. Work items are assigned to the persistent CTAs as in hgx_attn_forward
+ * (longest first, each to the least-loaded CTA).
  *
  * Arguments are those of hgx_attn_forward with the config in place of a handle (validated
  * on every call), plus `synchronize`: when nonzero the call waits for the stream and returns
  * HGX_ERR_TIMEOUT if a bounded device wait ran out; when zero it returns after the launches
  * and such a timeout goes unreported. The first call on each device looks up the device
  * address of the scratch array (cudaGetSymbolAddress, with that device current); make that
- * first call before any stream capture. All calls share the scratch and the host buffers,
- * which keep the previous call's contents (the error word is cleared at the start of each
- * call): calls that overlap on the GPU, or run from several host threads at once, race. */
+ * first call before any stream capture. The plan is uploaded with cudaMemcpyAsync from the
+ * library's static pageable host buffers (the driver stages each copy before the call
+ * returns, so the call may wait on the host). A call on a stream that is being captured
+ * (or on the legacy stream while another stream is captured) returns HGX_ERR_UNSUPPORTED
+ * before any device work: a recorded copy would read those shared host buffers again at
+ * replay, after later calls had rewritten them. All calls share the scratch and the host
+ * buffers, which keep the previous call's contents (the error word is cleared at the start
+ * of each call): calls that overlap on the GPU, or run from several host threads at once,
+ * race. */
 #define HGX_NOALLOC_MAX_TOKENS 16384
 #define HGX_NOALLOC_MAX_BATCH 64
 

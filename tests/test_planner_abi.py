@@ -9,6 +9,7 @@
 import ctypes
 import os
 import re
+import subprocess
 
 import numpy as np
 import pytest
@@ -162,11 +163,16 @@ def test_create_rejects_bad_configs():
 def _fake(addr):
     # a non-null host integer posing as a device pointer: these calls must fail before
     # anything dereferences it
-    class P:
-        def data_ptr(self):
-            return addr
+    return None if addr is None else ctypes.c_void_p(addr)
 
-    return P()
+
+def _c_call(a, name, ptrs, cu, segs, cu_segs, *tail):
+    """Calls a path entry point of the C ABI directly (below the binding's own tensor
+    checks) with raw pointers, raising HgxError like the binding does."""
+    c, sg, cs = B._descriptor(cu, segs, cu_segs)
+    extra = [B._ptr(B._i32(t).reshape(-1)) for t in tail]
+    st = getattr(B.lib(), name)(a.handle, None, *ptrs, len(c) - 1, B._ptr(c), B._ptr(sg), B._ptr(cs), *extra)
+    a._check(st, name)
 
 
 def test_forward_rejects_before_device_work():
@@ -175,29 +181,29 @@ def test_forward_rejects_before_device_work():
     good = [_fake(0x10000 * (i + 1)) for i in range(7)]
     # malformed descriptor
     with pytest.raises(B.HgxError) as e:
-        a.forward(*good, [0, 8], [[0, 7, 0]], [0, 1], stream=0)
+        _c_call(a, "hgx_attn_forward", good, [0, 8], [[0, 7, 0]], [0, 1])
     assert e.value.status == B.HGX_ERR_INVALID_ARG
     # null pointer
     for i in range(7):
         args = list(good)
         args[i] = None
         with pytest.raises(B.HgxError) as e:
-            a.forward(*args, cu, segs, cu_segs, stream=0)
+            _c_call(a, "hgx_attn_forward", args, cu, segs, cu_segs)
         assert e.value.status == B.HGX_ERR_INVALID_ARG
     # misaligned pointer
     args = list(good)
     args[2] = _fake(0x30008)
     with pytest.raises(B.HgxError) as e:
-        a.forward(*args, cu, segs, cu_segs, stream=0)
+        _c_call(a, "hgx_attn_forward", args, cu, segs, cu_segs)
     assert e.value.status == B.HGX_ERR_INVALID_ARG and "aligned" in str(e.value)
     # out overlapping q
     args = list(good)
     args[3] = _fake(0x10000 + 4096)
     with pytest.raises(B.HgxError) as e:
-        a.forward(*args, cu, segs, cu_segs, stream=0)
+        _c_call(a, "hgx_attn_forward", args, cu, segs, cu_segs)
     assert e.value.status == B.HGX_ERR_INVALID_ARG and "overlap" in str(e.value)
     # an empty batch returns OK without touching the device (works without a GPU)
-    a.forward(*[None] * 7, [0, 0], np.zeros((0, 3)), [0, 0], stream=0)
+    _c_call(a, "hgx_attn_forward", [None] * 7, [0, 0], np.zeros((0, 3)), [0, 0])
     a.close()
 
 
@@ -210,7 +216,7 @@ def test_forward_from_checks_the_reused_prefix_before_device_work():
     good = [_fake(0x40000000 * (i + 1)) for i in range(7)]
     for first, ok in ((0, True), (256, True), (257, True), (258, False), (8449, True), (-1, False), (8450, False)):
         try:
-            a.forward_from(*good, cu, segs, cu_segs, [first], stream=0)
+            _c_call(a, "hgx_attn_forward_from", good, cu, segs, cu_segs, [first])
             raised = None
         except B.HgxError as e:
             raised = e
@@ -240,6 +246,18 @@ def test_library_exports_every_declared_symbol():
     L = ctypes.CDLL(B.library_path)
     for name in declared:
         assert hasattr(L, name), name
+
+
+def test_header_declares_every_exported_symbol():
+    """The reverse direction: every hgx_* function the library exports has a prototype in
+    include/hgx_attn.h (the dynamic symbol table of the library built here, read with nm)."""
+    with open(os.path.join(ROOT, "include", "hgx_attn.h")) as f:
+        text = f.read()
+    declared = set(re.findall(r"\b(hgx_attn_\w+)\s*\(", text))
+    nm = subprocess.run(["nm", "-D", "--defined-only", B.library_path], capture_output=True, text=True, check=True)
+    exported = {ln.split()[-1] for ln in nm.stdout.splitlines() if ln.split() and ln.split()[-1].startswith("hgx_")}
+    assert exported, nm.stdout[:200]
+    assert exported <= declared, sorted(exported - declared)
 
 
 def test_binding_raises_without_library(monkeypatch, tmp_path):
@@ -274,3 +292,44 @@ def test_noalloc_rejects_before_device_work():
     assert _noalloc_status(bad, [0, 10], [[0, 10, 0]], [0, 1]) == B.HGX_ERR_INVALID_ARG
     # an empty batch is done without touching the device
     assert _noalloc_status(cfg, [0], np.zeros((0, 3)), [0]) == B.HGX_OK
+
+
+def test_binding_rejects_wrong_tensors_before_the_library():
+    """Marshalling checks of the binding (no GPU needed: every case is refused before any
+    pointer reaches the library): host tensors, wrong dtype, non-contiguous views and
+    wrong shapes raise INVALID_ARG."""
+    import torch
+
+    bf = torch.bfloat16
+    T = 5
+    ok = dict(q=torch.zeros(T, 32, 128, dtype=bf), k=torch.zeros(T, 8, 128, dtype=bf))
+    cases = [
+        ("host tensor", lambda: B._expect("q", ok["q"], "bf16", (32, 128), T)),
+        ("not a tensor", lambda: B._expect("q", np.zeros((T, 32, 128)), "bf16", (32, 128), T)),
+    ]
+    for what, fn in cases:
+        with pytest.raises(B.HgxError) as e:
+            fn()
+        assert e.value.status == B.HGX_ERR_INVALID_ARG, what
+
+    def check(t, dtype, tail, rows):  # CPU tensors that report is_cuda, so the later checks run here
+        orig = torch.Tensor.is_cuda
+        try:
+            torch.Tensor.is_cuda = property(lambda self: True)
+            B._expect("x", t, dtype, tail, rows)
+        finally:
+            torch.Tensor.is_cuda = orig
+
+    for what, t, dt, tail, rows in [
+        ("fp32", torch.zeros(T, 32, 128), "bf16", (32, 128), T),
+        ("int64 positions", torch.zeros(T, 3, dtype=torch.int64), "i32", (3,), T),
+        ("non-contiguous", torch.zeros(T, 128, 32, dtype=bf).transpose(1, 2), "bf16", (32, 128), T),
+        ("too few rows", torch.zeros(T - 1, 32, 128, dtype=bf), "bf16", (32, 128), T),
+        ("wrong heads", torch.zeros(T, 8, 128, dtype=bf), "bf16", (32, 128), T),
+        ("weight shape", torch.zeros(64, dtype=bf), "bf16", (128,), None),
+    ]:
+        with pytest.raises(B.HgxError) as e:
+            check(t, dt, tail, rows)
+        assert e.value.status == B.HGX_ERR_INVALID_ARG, what
+    check(torch.zeros(T + 2, 32, 128, dtype=bf), "bf16", (32, 128), T)  # more rows than needed is fine
+    check(torch.zeros(128, dtype=bf), "bf16", (128,), None)

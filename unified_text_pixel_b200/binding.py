@@ -138,6 +138,45 @@ def _dev_ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+def _expect(name, t, dtype, tail, rows):
+    """Marshalling check of one device tensor argument: a contiguous CUDA tensor of the
+    given dtype whose trailing dimensions are `tail` and that holds at least `rows` rows
+    (leading dimension; None = no leading dimension). Raises HgxError(INVALID_ARG)."""
+    import torch
+
+    if not isinstance(t, torch.Tensor):
+        raise HgxError(HGX_ERR_INVALID_ARG, f"{name}: expected a torch tensor, got {type(t).__name__}")
+    if not t.is_cuda:
+        raise HgxError(HGX_ERR_INVALID_ARG, f"{name}: must be a CUDA tensor (device {t.device})")
+    want = {"bf16": torch.bfloat16, "i32": torch.int32}[dtype]
+    if t.dtype != want:
+        raise HgxError(HGX_ERR_INVALID_ARG, f"{name}: dtype {t.dtype}, expected {want}")
+    if not t.is_contiguous():
+        raise HgxError(HGX_ERR_INVALID_ARG, f"{name}: must be contiguous (strides {tuple(t.stride())})")
+    shape = tuple(t.shape)
+    if rows is None:
+        ok = shape == tuple(tail)
+    else:
+        ok = len(shape) == 1 + len(tail) and shape[1:] == tuple(tail) and shape[0] >= rows
+    if not ok:
+        want_shape = list(tail) if rows is None else [f">={rows}", *tail]
+        raise HgxError(HGX_ERR_INVALID_ARG, f"{name}: shape {list(shape)}, expected {want_shape}")
+
+
+def _check_path(T, q=None, k=None, v=None, out=None, pos=None, wq=None, wk=None):
+    """Checks the tensors of the attention path for T packed tokens (nothing when T == 0:
+    the library then does no device work)."""
+    if T == 0:
+        return
+    for name, t, dt, tail in (("q", q, "bf16", (32, 128)), ("k", k, "bf16", (8, 128)), ("v", v, "bf16", (8, 128)),
+                              ("out", out, "bf16", (32, 128)), ("pos", pos, "i32", (3,))):
+        if t is not None:
+            _expect(name, t, dt, tail, T)
+    for name, t in (("wq", wq), ("wk", wk)):
+        if t is not None:
+            _expect(name, t, "bf16", (128,), None)
+
+
 def _stream_ptr(stream):
     """torch.cuda.Stream, a raw cudaStream_t integer, or None for torch's current stream."""
     if isinstance(stream, int):
@@ -192,6 +231,7 @@ class Attention:
     def forward(self, q, k, v, out, pos, wq, wk, cu_seqlens, segs, cu_segs, stream=None):
         """hgx_attn_forward: q, k overwritten with q', k'; out written."""
         cu, sg, cs = _descriptor(cu_seqlens, segs, cu_segs)
+        _check_path(int(cu[-1]) if cu.size else 0, q, k, v, out, pos, wq, wk)
         st = lib().hgx_attn_forward(self._h, _stream_ptr(stream), _dev_ptr(q), _dev_ptr(k), _dev_ptr(v),
                                     _dev_ptr(out), _dev_ptr(pos), _dev_ptr(wq), _dev_ptr(wk), len(cu) - 1,
                                     _ptr(cu), _ptr(sg), _ptr(cs))
@@ -200,6 +240,7 @@ class Attention:
     def forward_from(self, q, k, v, out, pos, wq, wk, cu_seqlens, segs, cu_segs, first_rows, stream=None):
         """hgx_attn_forward_from: recompute rows [first_rows[b], L_b) only (reused prefix)."""
         cu, sg, cs = _descriptor(cu_seqlens, segs, cu_segs)
+        _check_path(int(cu[-1]) if cu.size else 0, q, k, v, out, pos, wq, wk)
         fr = _i32(first_rows).reshape(-1)
         st = lib().hgx_attn_forward_from(self._h, _stream_ptr(stream), _dev_ptr(q), _dev_ptr(k), _dev_ptr(v),
                                          _dev_ptr(out), _dev_ptr(pos), _dev_ptr(wq), _dev_ptr(wk), len(cu) - 1,
@@ -208,12 +249,23 @@ class Attention:
 
     def qkv_projection(self, x, w_qkv, q, k, v, pos, wq, wk, stream=None):
         """q', k', v from x: tcgen05 GEMM with RMSNorm + rotation in its epilogue."""
+        T = int(x.shape[0])
+        if T:
+            _expect("x", x, "bf16", (4096,), T)
+            _expect("w_qkv", w_qkv, "bf16", (6144, 4096), None)
+        _check_path(T, q, k, v, None, pos, wq, wk)
         st = lib().hgx_attn_qkv_projection(self._h, _stream_ptr(stream), _dev_ptr(x), _dev_ptr(w_qkv), _dev_ptr(q),
                                            _dev_ptr(k), _dev_ptr(v), _dev_ptr(pos), _dev_ptr(wq), _dev_ptr(wk),
                                            int(x.shape[0]))
         self._check(st, "hgx_attn_qkv_projection")
 
     def out_projection(self, attn, w_o, y, stream=None):
+        """y = attn W_o^T (attn [T, 32, 128] or [T, 4096], w_o [4096, 4096], y [T, 4096])."""
+        T = int(attn.shape[0])
+        if T:
+            _expect("attn", attn, "bf16", (32, 128) if attn.dim() == 3 else (4096,), T)
+            _expect("w_o", w_o, "bf16", (4096, 4096), None)
+            _expect("y", y, "bf16", (4096,), T)
         st = lib().hgx_attn_out_projection(self._h, _stream_ptr(stream), _dev_ptr(attn), _dev_ptr(w_o), _dev_ptr(y),
                                            int(attn.shape[0]))
         self._check(st, "hgx_attn_out_projection")
@@ -221,6 +273,13 @@ class Attention:
     def layer_forward(self, x, w_qkv, w_o, q, k, v, attn, y, pos, wq, wk, cu_seqlens, segs, cu_segs, stream=None):
         """QKV projection (fused RMSNorm + rotation) -> masked attention -> output projection."""
         cu, sg, cs = _descriptor(cu_seqlens, segs, cu_segs)
+        T = int(cu[-1]) if cu.size else 0
+        if T:
+            _expect("x", x, "bf16", (4096,), T)
+            _expect("w_qkv", w_qkv, "bf16", (6144, 4096), None)
+            _expect("w_o", w_o, "bf16", (4096, 4096), None)
+            _expect("y", y, "bf16", (4096,), T)
+        _check_path(T, q, k, v, attn, pos, wq, wk)
         st = lib().hgx_attn_layer_forward(self._h, _stream_ptr(stream), _dev_ptr(x), _dev_ptr(w_qkv), _dev_ptr(w_o),
                                           _dev_ptr(q), _dev_ptr(k), _dev_ptr(v), _dev_ptr(attn), _dev_ptr(y),
                                           _dev_ptr(pos), _dev_ptr(wq), _dev_ptr(wk), len(cu) - 1, _ptr(cu),
@@ -229,12 +288,14 @@ class Attention:
 
     def prologue(self, q, k, pos, wq, wk, total_tokens=None, stream=None):
         T = q.shape[0] if total_tokens is None else total_tokens
+        _check_path(int(T), q, k, None, None, pos, wq, wk)
         st = lib().hgx_attn_prologue(self._h, _stream_ptr(stream), _dev_ptr(q), _dev_ptr(k), _dev_ptr(pos),
                                      _dev_ptr(wq), _dev_ptr(wk), int(T))
         self._check(st, "hgx_attn_prologue")
 
     def attention(self, q, k, v, out, cu_seqlens, segs, cu_segs, stream=None):
         cu, sg, cs = _descriptor(cu_seqlens, segs, cu_segs)
+        _check_path(int(cu[-1]) if cu.size else 0, q, k, v, out)
         st = lib().hgx_attn_attention(self._h, _stream_ptr(stream), _dev_ptr(q), _dev_ptr(k), _dev_ptr(v),
                                       _dev_ptr(out), len(cu) - 1, _ptr(cu), _ptr(sg), _ptr(cs))
         self._check(st, "hgx_attn_attention")

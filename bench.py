@@ -239,7 +239,7 @@ def run_reference(args):
         "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total_s / max(1, args.steps), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": _config_dict(w, None),
+        "config": _config_dict(w),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _blas_threads(), "kind": "oracle",
                          "cpu": _cpu_model(), "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -248,7 +248,7 @@ def run_reference(args):
     return 0
 
 
-def _config_dict(w, pairs):
+def _config_dict(w):
     segs = "; ".join(
         "+".join(f"{s.length}{'c' if s.kind == 0 else 'fs' if s.kind == 1 else 'fis'}" for s in b) for b in w.batches
     )
@@ -257,12 +257,65 @@ def _config_dict(w, pairs):
          "l2": f"inputs larger than L2: a distinct {48 * 128 * 2 * w.total_tokens / 1e6:.0f} MB "
                f"(q, k, v) input set per step",
          "parallelism": "replicas (one full workload per GPU)"}
-    if pairs is not None:
-        d["unmasked_gflop_per_step"] = round(pairs * FLOP_PER_PAIR / 1e9, 3)
     return d
 
 
 # ------------------------------------------------------------------------ GPU arm
+PER_WORKLOAD = ("hidream_tiny_321", "hidream_t2i_1024_cfg", "hidream_t2i_2048_cfg", "hidream_edit_2048",
+                "hunyuan_gca_9088", "hunyuan_multigen_9088")
+L2_FLUSH_BYTES = 256 << 20  # twice the 126 MB L2
+
+
+def per_workload_timings(H, a, peaks, iters=10, names=PER_WORKLOAD):
+    """Event-timed prologue and attention launches of every workload, each launch preceded by
+    a write of a buffer twice the size of L2 (outside the timed launch), on pristine q/k
+    restored before every prologue. Returns {name: figures}."""
+    import torch
+
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    res = {}
+    for name in names:
+        w = _workload(name)
+        cu, segs, cu_segs = _descriptor(w)
+        flops = _visible_pairs(w) * FLOP_PER_PAIR
+        T = w.total_tokens
+        host = W.tensors(w)
+        pristine = {n: host[n].cuda() for n in ("q", "k")}
+        d = {n: x.clone() for n, x in pristine.items()}
+        v, wq, wk = host["v"].cuda(), host["wq"].cuda(), host["wk"].cuda()
+        pos = torch.from_numpy(W.positions(w)).cuda()
+        out = torch.empty(T, 32, 128, dtype=torch.bfloat16, device="cuda")
+        pro, att = [], []
+        for i in range(iters + 2):
+            for n in d:
+                d[n].copy_(pristine[n])
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            flush.zero_()
+            ev[0].record(stream)
+            a.prologue(d["q"], d["k"], pos, wq, wk, stream=stream)
+            ev[1].record(stream)
+            flush.zero_()
+            ev[2].record(stream)
+            a.attention(d["q"], d["k"], v, out, cu, segs, cu_segs, stream=stream)
+            ev[3].record(stream)
+            torch.cuda.synchronize()
+            if i >= 2:
+                pro.append(ev[0].elapsed_time(ev[1]))
+                att.append(ev[2].elapsed_time(ev[3]))
+        if a.sync_status(stream) != H.HGX_OK:
+            raise RuntimeError(a.last_error())
+        att_ms, pro_ms = statistics.median(att), statistics.median(pro)
+        tf = flops / (att_ms * 1e-3) / 1e12
+        gbs = 80 * 128 * 2 * T / (pro_ms * 1e-3) / 1e9
+        res[name] = {"tokens": T, "unmasked_gflop": round(flops / 1e9, 3),
+                     "attention_ms": att_ms, "attention_tflops": tf, "attention_frac": tf / peaks["bf16_tflops"],
+                     "prologue_ms": pro_ms, "prologue_gbs": gbs, "prologue_frac": gbs / peaks["hbm_gbs"],
+                     "oracle_tflops": None}
+        del d, pristine, v, out
+    return res
+
+
 def run_gpu(args):
     import torch
 
@@ -421,7 +474,8 @@ def run_gpu(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": dict(_config_dict(w, pairs), **({"reuse_prefix_first_rows": first_rows} if first_rows else {})),
+        "config": dict(_config_dict(w), **({"reuse_prefix_first_rows": first_rows} if first_rows else {})),
+        "unmasked_gflop_per_step": round(flops / 1e9, 3),
         "pct_of_bf16_peak": 100.0 * value / ws / peak,
         "kernel_ms": {"prologue": pro_ms, "attention": att_ms} if not first_rows else
                      {"forward_from (prologue + attention)": att_ms},
@@ -455,12 +509,19 @@ def run_gpu(args):
         "clocks": clk.summary(),
     }
     del sets
+    if not args.no_per_workload and not first_rows:
+        _log("per-workload kernel timings")
+        line["per_workload"] = per_workload_timings(H, a, peaks)
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         _log("cpu baseline (oracle)")
         v, rows, secs, threads = cpu_oracle_sample(w, budget_s=args.cpu_seconds)
         line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                                 "cpu": _cpu_model(),
                                 "sample": f"{rows} random rows of {w.name} (all 32 query heads, fp64) in {secs:.1f} s"}
+        for name, r in line.get("per_workload", {}).items():
+            ov, orows, osecs, _ = cpu_oracle_sample(_workload(name), budget_s=args.cpu_seconds_per_workload)
+            r["oracle_tflops"] = ov
+            r["oracle_sample"] = f"{orows} random rows in {osecs:.1f} s on {threads} threads"
     a.close()
     if dist:
         dist.destroy_process_group()
@@ -558,7 +619,7 @@ def run_gpu_layer(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (random-init projection weights)",
-        "config": dict(_config_dict(w, _visible_pairs(w)), layer_gflop_per_step=round(flops / 1e9, 3),
+        "config": dict(_config_dict(w), layer_gflop_per_step=round(flops / 1e9, 3),
                        l2=f"inputs larger than L2: a distinct {x_bytes / 1e6:.0f} MB x per step"),
         "kernel_ms": {"qkv_projection": ms[0], "attention": ms[1], "out_projection": ms[2]},
         "roofline": dict(bound="tensor", kernel="attention_kernel", unit="TFLOP/s", peak=peak, traffic=None,
@@ -609,6 +670,9 @@ def main():
     p.add_argument("--cpu-seconds", type=float, default=15.0, help="budget of the CPU-baseline leg")
     p.add_argument("--ref-step-seconds", type=float, default=4.0, help="oracle seconds per reference step")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-per-workload", action="store_true", help="skip the per-workload kernel timings")
+    p.add_argument("--cpu-seconds-per-workload", type=float, default=2.0,
+                   help="oracle seconds per workload in the per-workload figures")
     p.add_argument("--layer", action="store_true",
                    help="time the whole attention layer (QKV projection, attention, output projection)")
     p.add_argument("--reuse-prefix", action="store_true",

@@ -1,12 +1,14 @@
-"""hgx_attn_forward_noalloc against hgx_attn_forward (GPU, through the C ABI).
+"""hgx_attn_forward_noalloc against hgx_attn_forward and the fp64 oracle (GPU, through
+the C ABI).
 
 The allocation-free entry point serves callers that may not allocate device memory (a
 framework that owns every byte through its own pool, a process whose footprint must not
 grow after start-up): it keeps its scratch in a fixed array inside the library. Its output
-must match the regular entry point's within the tolerance of the parity tests, on two calls
-in a row (the second call finds the first call's leftovers in the shared scratch). This
-file is collected last so that a run that stops at the first failure has already run
-every other test.
+must match the regular entry point's within the tolerance of the parity tests, on calls in
+a row (each later call finds the earlier calls' leftovers in the shared scratch), and the
+oracle's: element by element on the small workloads, on one row of every 64-token query
+block of the Hunyuan GCA workload (full_in_segment rows). This file is collected last so
+that a run that stops at the first failure has already run every other test.
 """
 import ctypes
 
@@ -14,6 +16,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle as O
 import workloads as W
 
 pytestmark = pytest.mark.gpu
@@ -59,7 +62,7 @@ def _h(a):
 
 def _noalloc(B, w):
     d = _inputs(w)
-    out = torch.empty_like(d["q"])
+    out = torch.full_like(d["q"], float("nan"))
     cfg = B.Attention.default_config()
     cu, segs, cu_segs = _desc(w)
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
@@ -72,7 +75,7 @@ def _noalloc(B, w):
 
 def _regular(B, w):
     d = _inputs(w)
-    out = torch.empty_like(d["q"])
+    out = torch.full_like(d["q"], float("nan"))
     a = B.Attention()
     a.forward(d["q"], d["k"], d["v"], out, d["pos"], d["wq"], d["wk"], *_desc(w))
     assert a.sync_status() == B.HGX_OK
@@ -80,14 +83,34 @@ def _regular(B, w):
     return out
 
 
+def _within(got, ref, what):
+    err = np.abs(got.astype(np.float64) - ref)
+    assert np.isfinite(got).all(), what
+    assert err.max() <= ATOL_MAX and err.mean() <= ATOL_MEAN, (what, float(err.max()), float(err.mean()))
+
+
+def _oracle_rows(w, rows):
+    t = W.tensors(w)
+    segs, cu_segs = W.flat_segments(w)
+    return O.attention_rows(t["q"], t["k"], t["v"], W.positions(w), t["wq"], t["wk"], W.cu_seqlens(w), segs,
+                            cu_segs, rows)
+
+
 def test_noalloc_matches_forward_on_two_calls_in_a_row(lib):
     B = lib
-    for w in (W.config(1), W.config(0)):  # the second call reuses the first call's scratch
+    # the Hunyuan GCA workload (full_in_segment image rows, 9088 tokens), then the 1024^2 CFG
+    # pair and the tiny layout: each later call reuses the earlier calls' scratch
+    for w in (W.config(4), W.config(1), W.config(0)):
         got = _noalloc(B, w).float().cpu().numpy()
         ref = _regular(B, w).float().cpu().numpy()
-        err = np.abs(got - ref)
-        assert np.isfinite(got).all()
-        assert err.max() <= ATOL_MAX and err.mean() <= ATOL_MEAN, (w.name, float(err.max()), float(err.mean()))
+        _within(got, ref, w.name + " vs hgx_attn_forward")
+        if w.total_tokens <= 2200:
+            rows = list(range(w.total_tokens))
+        else:
+            rng = np.random.default_rng(4)
+            rows = sorted({int(rng.integers(r0, min(w.total_tokens, r0 + 64))) for r0 in range(0, w.total_tokens, 64)}
+                          | {511, 512, 4607, 4608, 4863, 4864, w.total_tokens - 1})
+        _within(got[rows], _oracle_rows(w, rows), w.name + " vs oracle")
 
 
 def test_noalloc_rejects_sizes_beyond_its_limit(lib):
@@ -101,3 +124,30 @@ def test_noalloc_rejects_sizes_beyond_its_limit(lib):
     st = B.lib().hgx_attn_forward_noalloc(ctypes.byref(cfg), None, z, z, z, z, z, z, z, 1, _h(cu), _h(segs),
                                           _h(cu_segs), 1)
     assert st == B.HGX_ERR_UNSUPPORTED
+
+
+def test_noalloc_refuses_a_capturing_stream(lib):
+    """The plan is uploaded from the library's shared static host buffers, which a recorded
+    copy would read again at replay; so a call on a stream under capture returns
+    HGX_ERR_UNSUPPORTED before any device work, and the next ordinary call still matches."""
+    B = lib
+    w = W.config(0)
+    d = _inputs(w)
+    out = torch.full_like(d["q"], float("nan"))
+    cfg = B.Attention.default_config()
+    cu, segs, cu_segs = _desc(w)
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    statuses = []
+    with torch.cuda.graph(g, stream=side):  # side is the current (capturing) stream in here
+        sp = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        statuses.append(B.lib().hgx_attn_forward_noalloc(
+            ctypes.byref(cfg), sp, _p(d["q"]), _p(d["k"]), _p(d["v"]), _p(out), _p(d["pos"]), _p(d["wq"]),
+            _p(d["wk"]), len(cu) - 1, _h(cu), _h(segs), _h(cu_segs), 0))
+        out.add_(0)  # keeps the capture non-empty; the graph is never replayed
+    assert statuses == [B.HGX_ERR_UNSUPPORTED]
+    torch.cuda.synchronize()
+    assert torch.isnan(out).all()  # nothing ran
+    got = _noalloc(B, w).float().cpu().numpy()
+    ref = _regular(B, w).float().cpu().numpy()
+    _within(got, ref, "after a refused capture")

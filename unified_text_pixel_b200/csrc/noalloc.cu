@@ -10,7 +10,7 @@
 //
 // Where the scratch lives instead: the attention kernel needs, besides its inputs and
 // outputs, the per-row key limits, the work list and a device error word. Here they sit
-// in one file-scope __device__ array of fixed size (kScratchBytes, about 145 KB), which
+// in one file-scope __device__ array of fixed size (kScratchBytes, about 185 KB), which
 // every GPU that loads this library holds until the process exits. The array's name in
 // host code is only a host-side stand-in, so the device address is looked up once per
 // device with cudaGetSymbolAddress (done by the first call on that device, with the device
@@ -18,9 +18,17 @@
 // of the same fixed size.
 //
 // Sharing: every call uses the same arrays, which keep the last call's contents. The error
-// word is cleared at the start of each call; the limits and the work list are fully
-// rewritten. Calls that overlap on the GPU (on different streams) race on the scratch, and
-// calls from several host threads at once race on the host buffers: serialise them.
+// word is cleared at the start of each call; the limits, the work list and the CTA
+// offsets are fully rewritten. Calls that overlap on the GPU (on different streams) race
+// on the scratch, and calls from several host threads at once race on the host buffers:
+// serialise them. The plan is uploaded with cudaMemcpyAsync from the static (pageable)
+// host buffers; the driver stages such a copy before the call returns, so the next call
+// may rewrite the buffers, but a replay of a recorded copy would read whatever they hold
+// then -- which is why a call on a stream that is being captured is refused.
+//
+// Work assignment: as in the handle path, every persistent CTA gets a contiguous list of
+// items, each item (longest first) going to the least-loaded CTA; the heap of CTA loads
+// lives in a fixed static array.
 //
 // The paper has no counterpart to this entry point; it exists for the callers above.
 #include <cuda.h>
@@ -41,11 +49,13 @@ constexpr int32_t kMaxKvHeads = 8;
 // query blocks: sum over elements of ceil(L_b / 64) <= T / 64 + batch
 constexpr int32_t kMaxItems = kMaxKvHeads * (kMaxTokens / hgx::kBlockTokens + kMaxBatch);
 constexpr int32_t kMaxKeyBlocks = kMaxTokens / hgx::kBlockKeys;
+constexpr int32_t kMaxCtas = 256;  // persistent CTAs (one per SM; B200 has 148)
 
 constexpr size_t kErrOffset = 0;
 constexpr size_t kLimOffset = 256;
 constexpr size_t kItemsOffset = kLimOffset + sizeof(int32_t) * kMaxTokens;
-constexpr size_t kScratchBytes = kItemsOffset + sizeof(hgx::WorkItem) * kMaxItems;
+constexpr size_t kCtaOffsetsOffset = kItemsOffset + sizeof(hgx::WorkItem) * kMaxItems;
+constexpr size_t kScratchBytes = kCtaOffsetsOffset + sizeof(int32_t) * (kMaxCtas + 1);
 
 // device scratch shared by every call (see the file comment)
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
@@ -55,6 +65,11 @@ static int32_t s_lim[kMaxTokens];
 static hgx::WorkItem s_unsorted[kMaxItems];
 static hgx::WorkItem s_items[kMaxItems];
 static int32_t s_bucket[kMaxKeyBlocks + 2];
+static hgx::WorkItem s_assigned[kMaxItems];
+static int32_t s_owner[kMaxItems];
+static int32_t s_cta_offsets[kMaxCtas + 1];
+static int64_t s_heap_load[kMaxCtas];
+static int32_t s_heap_cta[kMaxCtas];
 
 struct DeviceSetup {
   unsigned char* scratch = nullptr;  // device address of g_noalloc_scratch
@@ -128,10 +143,65 @@ hgx_status check_config(const hgx_attn_config* cfg) {
     if (cfg->mrope_section[i] < 0) return HGX_ERR_INVALID_ARG;
   if (cfg->rope_layout < HGX_ROPE_MROPE_INTERLEAVED || cfg->rope_layout > HGX_ROPE_2D_HALVES)
     return HGX_ERR_INVALID_ARG;
-  if (cfg->rope_layout == HGX_ROPE_MROPE_INTERLEAVED &&
-      cfg->mrope_section[0] + cfg->mrope_section[1] + cfg->mrope_section[2] != 64)
-    return HGX_ERR_INVALID_ARG;
+  if (cfg->rope_layout == HGX_ROPE_MROPE_INTERLEAVED) {
+    if (cfg->mrope_section[0] + cfg->mrope_section[1] + cfg->mrope_section[2] != 64)
+      return HGX_ERR_INVALID_ARG;
+    // the interleaved assignment must give each axis exactly its section's count
+    double inv[64];
+    int32_t axis[64], count[3] = {0, 0, 0};
+    hgx::mrope_tables(cfg->rope_theta, cfg->head_dim, cfg->mrope_section, cfg->rope_layout, inv, axis);
+    for (int i = 0; i < 64; ++i) ++count[axis[i]];
+    for (int i = 0; i < 3; ++i)
+      if (count[i] != cfg->mrope_section[i]) return HGX_ERR_UNSUPPORTED;
+  }
   return HGX_OK;
+}
+
+// Min-heap of (load, cta) pairs over the static arrays: the least-loaded CTA, ties to the
+// lower index.
+bool heap_less(int32_t a, int32_t b) {
+  return s_heap_load[a] < s_heap_load[b] || (s_heap_load[a] == s_heap_load[b] && s_heap_cta[a] < s_heap_cta[b]);
+}
+void heap_swap(int32_t a, int32_t b) {
+  const int64_t l = s_heap_load[a];
+  s_heap_load[a] = s_heap_load[b];
+  s_heap_load[b] = l;
+  const int32_t c = s_heap_cta[a];
+  s_heap_cta[a] = s_heap_cta[b];
+  s_heap_cta[b] = c;
+}
+void heap_sift_down(int32_t n) {
+  for (int32_t i = 0;;) {
+    const int32_t l = 2 * i + 1, r = l + 1;
+    int32_t m = i;
+    if (l < n && heap_less(l, m)) m = l;
+    if (r < n && heap_less(r, m)) m = r;
+    if (m == i) return;
+    heap_swap(i, m);
+    i = m;
+  }
+}
+
+// Longest-processing-time assignment of the n sorted items of s_items to `grid` CTAs
+// (cost of an item: its key blocks plus 2 for loading Q and writing O). Fills
+// s_cta_offsets[0..grid] and reorders the items into s_assigned so that every CTA's list is
+// contiguous and keeps the longest-first order.
+void assign(int32_t n, int32_t grid) {
+  for (int32_t c = 0; c < grid; ++c) {  // all loads 0: the index order is a valid heap
+    s_heap_load[c] = 0;
+    s_heap_cta[c] = c;
+  }
+  for (int32_t c = 0; c <= grid; ++c) s_cta_offsets[c] = 0;
+  for (int32_t i = 0; i < n; ++i) {
+    const int32_t c = s_heap_cta[0];
+    s_owner[i] = c;
+    ++s_cta_offsets[c + 1];
+    s_heap_load[0] += s_items[i].n_total + 2;
+    heap_sift_down(grid);
+  }
+  for (int32_t c = 0; c < grid; ++c) s_cta_offsets[c + 1] += s_cta_offsets[c];
+  for (int32_t c = 0; c < grid; ++c) s_heap_cta[c] = s_cta_offsets[c];  // next free slot per CTA
+  for (int32_t i = 0; i < n; ++i) s_assigned[s_heap_cta[s_owner[i]]++] = s_items[i];
 }
 
 // Validates the descriptor and plans into the static host buffers. Returns the number of
@@ -212,6 +282,7 @@ extern "C" hgx_status hgx_attn_forward_noalloc(const hgx_attn_config* cfg, void*
                                                const int32_t* cu_segs_host, int32_t synchronize) {
   hgx_status st = check_config(cfg);
   if (st != HGX_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
   int32_t T = 0, n_items = 0;
   if ((st = plan(batch, cu_seqlens_host, segs_host, cu_segs_host, &T, &n_items)) != HGX_OK)
     return st;
@@ -222,19 +293,34 @@ extern "C" hgx_status hgx_attn_forward_noalloc(const hgx_attn_config* cfg, void*
   const size_t qb = size_t(T) * 8192, kb = size_t(T) * 2048;
   if (overlaps(out, qb, q, qb) || overlaps(out, qb, k, kb) || overlaps(out, qb, v, kb))
     return HGX_ERR_INVALID_ARG;
+  {
+    // refused while the stream is being captured (see the file comment); the legacy
+    // stream under another stream's capture reports cudaErrorStreamCaptureImplicit
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    const cudaError_t e = cudaStreamIsCapturing(s, &cs);
+    if (e == cudaErrorStreamCaptureImplicit || (e == cudaSuccess && cs != cudaStreamCaptureStatusNone))
+      return HGX_ERR_UNSUPPORTED;
+    if (e != cudaSuccess) return HGX_ERR_CUDA;
+  }
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return HGX_ERR_CUDA;
   if ((st = setup_device(dev)) != HGX_OK) return st;
   const DeviceSetup& d = s_dev[dev];
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int32_t grid = n_items < d.num_sms ? (n_items < kMaxCtas ? n_items : kMaxCtas)
+                                            : (d.num_sms < kMaxCtas ? d.num_sms : kMaxCtas);
+  assign(n_items, grid);
 
   uint32_t* d_err = reinterpret_cast<uint32_t*>(d.scratch + kErrOffset);
   int32_t* d_lim = reinterpret_cast<int32_t*>(d.scratch + kLimOffset);
   hgx::WorkItem* d_items = reinterpret_cast<hgx::WorkItem*>(d.scratch + kItemsOffset);
-  // the error word must start at zero; limits and work list are rewritten in full
+  int32_t* d_cta_offsets = reinterpret_cast<int32_t*>(d.scratch + kCtaOffsetsOffset);
+  // the error word must start at zero; limits, work list and CTA offsets are rewritten in
+  // full
   if (cudaMemsetAsync(d_err, 0, sizeof(uint32_t), s) != cudaSuccess ||
       cudaMemcpyAsync(d_lim, s_lim, sizeof(int32_t) * T, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(d_items, s_items, sizeof(hgx::WorkItem) * n_items, cudaMemcpyHostToDevice, s) !=
+      cudaMemcpyAsync(d_items, s_assigned, sizeof(hgx::WorkItem) * n_items, cudaMemcpyHostToDevice, s) !=
+          cudaSuccess ||
+      cudaMemcpyAsync(d_cta_offsets, s_cta_offsets, sizeof(int32_t) * (grid + 1), cudaMemcpyHostToDevice, s) !=
           cudaSuccess)
     return HGX_ERR_CUDA;
 
@@ -242,14 +328,7 @@ extern "C" hgx_status hgx_attn_forward_noalloc(const hgx_attn_config* cfg, void*
   int32_t axis[64];
   hgx::mrope_tables(cfg->rope_theta, cfg->head_dim, cfg->mrope_section, cfg->rope_layout,
                     rope.inv_freq, axis);
-  int32_t count[3] = {0, 0, 0};
-  for (int i = 0; i < 64; ++i) {
-    rope.axis[i] = static_cast<uint8_t>(axis[i]);
-    ++count[axis[i]];
-  }
-  if (cfg->rope_layout == HGX_ROPE_MROPE_INTERLEAVED)
-    for (int i = 0; i < 3; ++i)
-      if (count[i] != cfg->mrope_section[i]) return HGX_ERR_UNSUPPORTED;
+  for (int i = 0; i < 64; ++i) rope.axis[i] = static_cast<uint8_t>(axis[i]);
   if (hgx::launch_prologue(s, q, k, pos_thw, q_norm_w, k_norm_w, T, cfg->rms_eps, rope) != cudaSuccess)
     return HGX_ERR_CUDA;
 
@@ -262,6 +341,7 @@ extern "C" hgx_status hgx_attn_forward_noalloc(const hgx_attn_config* cfg, void*
   hgx::AttnParams p{};
   p.items = d_items;
   p.n_items = n_items;
+  p.cta_offsets = d_cta_offsets;
   p.total_tokens = T;
   p.lim = d_lim;
   p.out = out;
@@ -269,7 +349,6 @@ extern "C" hgx_status hgx_attn_forward_noalloc(const hgx_attn_config* cfg, void*
   p.flags = 0;
   p.err = d_err;
   p.wait_limit_ns = 2000000000ull;
-  const int grid = n_items < d.num_sms ? n_items : d.num_sms;
   if (hgx::launch_attention(s, mq, mk, mv, p, grid) != cudaSuccess) return HGX_ERR_CUDA;
   if (!synchronize) return HGX_OK;
   if (cudaStreamSynchronize(s) != cudaSuccess) return HGX_ERR_CUDA;

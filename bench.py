@@ -92,6 +92,19 @@ def _descriptor(w):
     return W.cu_seqlens(w), segs, cu_segs
 
 
+def _has_splits(w, first_rows=None):
+    """Whether the library's planner splits items of this workload on this GPU (then a combine
+    kernel follows the attention kernel)."""
+    import torch
+
+    import unified_text_pixel_b200 as H
+
+    if first_rows:
+        return False  # reuse plans are scheduled like full ones; counted without a combine
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    return bool((H.schedule(*_descriptor(w), sms)[:, 5] >= 0).any())
+
+
 def _visible_pairs(w):
     # the product's own planner (host side of the library)
     import unified_text_pixel_b200 as H
@@ -504,8 +517,10 @@ def run_gpu(args):
                        "overlapping neighbouring steps' forwards"},
         "exp_offload": "none: MUFU ex2.approx for every score (a polynomial exp2 on the FMA pipe "
                        "for part of the scores measured slower on B200)",
+        # per step: the prologue launches, the attention kernel and, when the planner split
+        # items, the combine kernel
         "gpu_launches": (1 + (sum(1 for b in range(len(w.batches)) if first_rows[b] < w.lengths[b])
-                              if first_rows else 1)) * args.steps,
+                              if first_rows else 1) + (1 if _has_splits(w, first_rows) else 0)) * args.steps,
         "clocks": clk.summary(),
     }
     del sets
@@ -625,7 +640,8 @@ def run_gpu_layer(args):
         "roofline": dict(bound="tensor", kernel="attention_kernel", unit="TFLOP/s", peak=peak, traffic=None,
                          peak_source=f"{peak_src} bf16 dense (burst)", **roof(att_flops, ms[1])),
         "gemm_roofline": {"qkv_projection": roof(qkv_flops, ms[0]), "out_projection": roof(out_flops, ms[2])},
-        "gpu_launches": 4 * args.steps,
+        # per step: rotation table, QKV GEMM, attention (+ combine when items are split), output GEMM
+        "gpu_launches": (4 + (1 if _has_splits(w) else 0)) * args.steps,
         "clocks": clk.summary(),
     }
     a.close()

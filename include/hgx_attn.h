@@ -241,6 +241,22 @@ hgx_status hgx_attn_visible_pairs(int32_t batch, const int32_t* cu_seqlens_host,
                                   const hgx_segment* segs_host, const int32_t* cu_segs_host,
                                   uint64_t* pairs);
 
+/* Host only. The schedule of the attention kernel's persistent CTAs for this descriptor on
+ * `ctas` CTAs (the library uses the device's SM count), for tests and tools: 8 int32 per
+ * work item in execution order, (cta, q0, kv_head, kb0, n_total, part, n_full, list_off).
+ * A work item covers 64 query tokens x the 4 query heads of one KV head; it processes key
+ * blocks kb0 .. kb0 + n_total - 1 (prefix form, list_off < 0) or the n_total blocks of its
+ * key-block list (list form). part >= 0 marks one of the two halves of a split item, which
+ * write partial results that a combine kernel merges. mode 0: the library's own policy;
+ * 1: the wrap-around schedule with split items is taken whenever its makespan plus the
+ * combine's cost is smaller; 2: as under HGX_DEBUG_SPLIT_TEST (every prefix-form item of
+ * two or more key blocks split in two). out has room for cap items (8 int32 each);
+ * *n_items receives the count; out may be NULL to query the count. */
+hgx_status hgx_attn_schedule(int32_t batch, const int32_t* cu_seqlens_host,
+                             const hgx_segment* segs_host, const int32_t* cu_segs_host,
+                             int32_t ctas, int32_t mode, int32_t* out, size_t cap,
+                             size_t* n_items);
+
 /* Synchronizes `stream`, then reads and clears the handle's device error word: returns
  * HGX_ERR_TIMEOUT if a bounded wait ran out since the last check, HGX_ERR_CUDA if the
  * stream reports an error, HGX_OK otherwise. */
@@ -253,6 +269,9 @@ hgx_status hgx_attn_sync_status(hgx_attn_handle* h, void* stream);
 #define HGX_DEBUG_FAIL_ALLOC 4u /* the next device allocation of the planner scratch reports
                                    HGX_ERR_OOM instead of allocating (one-shot: the flag
                                    clears itself); nothing is launched by that call */
+#define HGX_DEBUG_SPLIT_TEST 8u /* the planner splits every prefix-form work item of two or
+                                   more key blocks into two halves by key blocks (exercises
+                                   the split path and its combine kernel on any input) */
 
 /* Sets debug flags and the bound of every device wait in nanoseconds (0 keeps the
  * default of 2 s). The HGX_DEBUG environment variable (an integer) sets the initial
@@ -267,7 +286,7 @@ hgx_status hgx_attn_set_debug(hgx_attn_handle* h, uint32_t flags, uint64_t wait_
  * one allocates) and calls no cudaMalloc, cudaFree, cudaMallocHost or heap allocation.
  *
  * Scratch (per-row key limits, work list, per-CTA item offsets, error word) lives in one
- * fixed-size device array inside the library (about 145 KB, held by every GPU that loads
+ * fixed-size device array inside the library (about 185 KB, held by every GPU that loads
  * the library until the process exits); planning uses fixed-size static host buffers. Hence
  * the limits: at most HGX_NOALLOC_MAX_TOKENS packed tokens and HGX_NOALLOC_MAX_BATCH batch
  * elements, and no gen_image segments; other requests return HGX_ERR_UNSUPPORTED before

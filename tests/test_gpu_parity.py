@@ -6,9 +6,13 @@ q'/k' within bf16 rounding of the fp64 values (relative 2^-8 plus 1e-5 absolute 
 fp32 arithmetic before rounding).
 
 Small configurations are compared element by element on every output; the full-size
-workloads (2048^2 text-to-image and edit, Hunyuan GCA) run in exactly the launch
-configuration the benchmark times and are compared on sampled rows that the oracle
-computes one by one (segment boundaries, tile edges, first and last rows, random rows).
+workloads (2048^2 text-to-image and edit, Hunyuan GCA, the multi-Gen-Image training mask)
+run in exactly the launch configuration the benchmark times and are compared on sampled
+rows that the oracle computes one by one: one random row of every 64-token query block of
+every batch element (each block is one work item per KV head, and a row covers all 32
+query heads, so every work item is checked), plus segment boundaries, tile edges, first and
+last rows. The output buffer is filled with NaN before every call and must come back
+finite everywhere, so a work item that is dropped or written to the wrong rows fails.
 """
 import numpy as np
 import pytest
@@ -49,11 +53,16 @@ def _device_inputs(w):
     return t, d
 
 
+def _nan_like(x):
+    return torch.full_like(x, float("nan"))
+
+
 def _run(hgx, w, d=None):
+    """hgx_attn_forward into an output prefilled with NaN (rows it does not write stay NaN)."""
     H, a = hgx
     if d is None:
         _, d = _device_inputs(w)
-    out = torch.empty_like(d["q"])
+    out = _nan_like(d["q"])
     a.forward(d["q"], d["k"], d["v"], out, d["pos"], d["wq"], d["wk"], *_desc(w))
     assert a.sync_status() == H.HGX_OK
     return out, d
@@ -150,11 +159,7 @@ def test_forward_multigen_full_size_sampled_rows(hgx):
     w = W.CONFIG_BY_NAME["hunyuan_multigen_9088"]
     t, _ = _device_inputs(w)
     out, _ = _run(hgx, w)
-    rows = _sample_rows(w, seed=9)
-    segs, cu_segs = W.flat_segments(w)
-    ref = O.attention_rows(t["q"], t["k"], t["v"], W.positions(w), t["wq"], t["wk"], W.cu_seqlens(w), segs,
-                           cu_segs, rows)
-    _compare(out[rows].float().cpu().numpy(), ref, w.name)
+    _check_sampled(w, t, out, seed=9)
 
 
 def test_attention_alone_on_kernel_rotated_inputs(hgx):
@@ -215,19 +220,24 @@ def test_online_rescale_path_with_divergent_rows(hgx):
 
 def test_forward_from_reuses_the_text_prefix(hgx):
     """A denoising step that keeps the text before <|tms|> (causal, so unchanged across
-    steps) and recomputes the rest: bit-identical to a full forward on the same inputs, and
-    the reused output rows are left untouched."""
+    steps: model card, "What this model is" and "Performance") and recomputes the rest.
+    The whole step-1 output is compared element by element with the fp64 oracle on the
+    step-1 inputs (the reused rows come from step 0, whose inputs they share); in addition
+    the recomputed rows are bit-identical to a full forward on the same inputs, the reused
+    output rows are left untouched and the recomputed k rows are rotated like a full
+    prologue."""
     H, a = hgx
     w = W.config(1)  # CFG pair: (128 text + <|tms|>, 1024 patches), (16 text + <|tms|>, 1024)
     cu, segs, cu_segs = _desc(w)
     first = [128, 16]
     t0 = W.tensors(w)
     t1 = W.tensors(W.Workload(w.name, w.batches, seed=w.seed + 100, style=w.style))
-    pos = torch.from_numpy(W.positions(w)).cuda()
+    pos_h = W.positions(w)
+    pos = torch.from_numpy(pos_h).cuda()
     wq, wk = t0["wq"].cuda(), t0["wk"].cuda()
     # step 0: full forward; k is rotated in place
     q0, k0, v0 = t0["q"].cuda(), t0["k"].cuda(), t0["v"].cuda()
-    out0 = torch.empty_like(q0)
+    out0 = _nan_like(q0)
     a.forward(q0, k0, v0, out0, pos, wq, wk, cu, segs, cu_segs)
     suffix = torch.zeros(w.total_tokens, dtype=torch.bool)
     for b in range(len(cu) - 1):
@@ -240,9 +250,16 @@ def test_forward_from_reuses_the_text_prefix(hgx):
     out1 = out0.clone()
     a.forward_from(q1, k1, v1, out1, pos, wq, wk, cu, segs, cu_segs, first)
     assert a.sync_status() == H.HGX_OK
-    # the same step computed from scratch
+    # against the oracle on the step-1 inputs (raw q, k, v: prefix from step 0, suffix new)
+    ref, _, kp_ref = O.forward(mix(t1["q"], t0["q"]), mix(t1["k"], t0["k"]), mix(t1["v"], t0["v"]), pos_h, t0["wq"],
+                               t0["wk"], cu, segs, cu_segs)
+    got = out1.float().cpu().numpy()
+    _compare(got, ref, "forward_from vs oracle")
+    _compare(got[suffix.numpy()], ref[suffix.numpy()], "recomputed rows vs oracle")
+    np.testing.assert_allclose(k1.float().cpu().numpy(), kp_ref, rtol=2.0 ** -8, atol=1e-5)
+    # the same step computed from scratch by the full path
     qr, kr, vr = mix(t1["q"], t0["q"]).cuda(), mix(t1["k"], t0["k"]).cuda(), mix(t1["v"], t0["v"]).cuda()
-    out_r = torch.empty_like(qr)
+    out_r = _nan_like(qr)
     a.forward(qr, kr, vr, out_r, pos, wq, wk, cu, segs, cu_segs)
     assert a.sync_status() == H.HGX_OK
     assert torch.equal(out1, out_r)
@@ -261,10 +278,17 @@ def test_single_token_returns_its_value(hgx):
 
 
 def _sample_rows(w, n_random=24, seed=0):
+    """Rows for the sampled full-size checks: one random row of every 64-token query block
+    of every batch element (so every work item of the kernel is checked on one of its
+    rows, for all 32 query heads), the rows around every segment boundary, the edges of
+    128-key blocks every 2048 tokens, first and last rows, and n_random rows anywhere."""
     rows = set()
     cu = W.cu_seqlens(w)
+    rng = np.random.default_rng(seed)
     for b, batch in enumerate(w.batches):
         base, L = int(cu[b]), w.lengths[b]
+        for r0 in range(0, L, 64):
+            rows.add(base + int(rng.integers(r0, min(L, r0 + 64))))
         for s in batch:
             for r in (s.start - 1, s.start, s.start + 1, s.start + s.length - 1):
                 if 0 <= r < L:
@@ -274,9 +298,22 @@ def _sample_rows(w, n_random=24, seed=0):
                 if 0 <= r < L:
                     rows.add(base + r)
         rows.update({base, base + L - 1})
-    rng = np.random.default_rng(seed)
     rows.update(int(x) for x in rng.integers(0, w.total_tokens, size=n_random))
     return sorted(rows)
+
+
+def _check_sampled(w, t, out, seed):
+    """Every row written (finite: the buffer was NaN-filled) and the sampled rows within
+    the tolerance of the oracle."""
+    assert torch.isfinite(out).all(), f"{w.name}: rows left unwritten"
+    rows = _sample_rows(w, seed=seed)
+    blocks = {(b, (r - int(W.cu_seqlens(w)[b])) // 64) for r in rows
+              for b in [int(np.searchsorted(W.cu_seqlens(w), r, side="right") - 1)]}
+    assert len(blocks) == sum(-(-L // 64) for L in w.lengths)  # every query block sampled
+    segs, cu_segs = W.flat_segments(w)
+    ref = O.attention_rows(t["q"], t["k"], t["v"], W.positions(w), t["wq"], t["wk"], W.cu_seqlens(w), segs,
+                           cu_segs, rows)
+    return _compare(out[rows].float().cpu().numpy(), ref, w.name)
 
 
 @pytest.mark.parametrize("cfg", [2, 3, 4])
@@ -284,17 +321,12 @@ def test_forward_full_size_sampled_rows(hgx, cfg):
     w = W.config(cfg)
     t, _ = _device_inputs(w)
     out, _ = _run(hgx, w)
-    rows = _sample_rows(w, seed=cfg)
-    segs, cu_segs = W.flat_segments(w)
-    ref = O.attention_rows(t["q"], t["k"], t["v"], W.positions(w), t["wq"], t["wk"], W.cu_seqlens(w), segs,
-                           cu_segs, rows)
-    got = out[rows].float().cpu().numpy()
-    _compare(got, ref, w.name)
-    assert torch.isfinite(out.float()).all()
+    _check_sampled(w, t, out, seed=cfg)
 
 
-def test_forward_is_deterministic(hgx):
-    w = W.config(1)
+@pytest.mark.parametrize("cfg", [1, 3])
+def test_forward_is_deterministic(hgx, cfg):
+    w = W.config(cfg)
     _, d0 = _device_inputs(w)
     _, d1 = _device_inputs(w)
     o0, _ = _run(hgx, w, d0)
@@ -316,25 +348,38 @@ def test_output_canaries_untouched(hgx):
 
 def test_maximum_token_count_sampled(hgx):
     """The largest packed size the ABI accepts (2^19 - 1 tokens, 128 batch elements):
-    exercises the highest byte offsets; sampled rows of the last elements."""
+    exercises the highest byte offsets. Every element carries the same q, k, v (a
+    4096-token draw, the last element its first 4095 tokens) and one of two segment
+    layouts, so every element must reproduce, bit for bit, the first element of its layout:
+    with the output NaN-filled, a dropped or misplaced work item anywhere fails. The first
+    element of each layout and the last element are checked against the oracle on one
+    random row of every 64-token query block."""
     H, a = hgx
     n_el, per = 128, 4096
     total = (1 << 19) - 1
     lens = [per] * (n_el - 1) + [total - per * (n_el - 1)]
-    batches = []
-    for i, L in enumerate(lens):
-        kinds = [(L // 4, W.CAUSAL), (L // 2, [W.FULL_SEQUENCE, W.FULL_IN_SEGMENT][i % 2]),
-                 (L - L // 4 - L // 2, W.CAUSAL)]
-        batches.append(kinds)
+    layouts = [[(per // 4, W.CAUSAL), (per // 2, kd), (per - per // 4 - per // 2, W.CAUSAL)]
+               for kd in (W.FULL_SEQUENCE, W.FULL_IN_SEGMENT)]
+    last = [(per // 4, W.CAUSAL), (per // 2, W.FULL_SEQUENCE), (lens[-1] - per // 4 - per // 2, W.CAUSAL)]
+    batches = [layouts[i % 2] for i in range(n_el - 1)] + [last]
     w = W.custom("max_tokens", batches, seed=21)
     assert w.total_tokens == total
-    t, _ = _device_inputs(w)
-    out, _ = _run(hgx, w)
-    cu = W.cu_seqlens(w)
-    rows = [int(cu[-2]) + r for r in (0, 1, 1023, 1024, 3000, lens[-1] - 1)] + [int(cu[60]) + 5, total - 1]
-    segs, cu_segs = W.flat_segments(w)
-    ref = O.attention_rows(t["q"], t["k"], t["v"], W.positions(w), t["wq"], t["wk"], cu, segs, cu_segs, rows)
-    _compare(out[rows].float().cpu().numpy(), ref, "max_tokens")
+    one = W.tensors(W.custom("max_el", [layouts[0]], seed=21))
+    dev = {n: one[n].cuda() for n in ("q", "k", "v")}
+    big = {n: x.repeat(n_el, 1, 1)[:total] for n, x in dev.items()}
+    del dev
+    big["pos"] = torch.from_numpy(W.positions(w)).cuda()
+    big["wq"], big["wk"] = one["wq"].cuda(), one["wk"].cuda()
+    out, _ = _run(hgx, w, big)
+    del big
+    assert torch.isfinite(out).all(), "rows left unwritten"
+    for i in range(2, n_el - 1):
+        assert torch.equal(out[i * per:(i + 1) * per], out[(i % 2) * per:(i % 2 + 1) * per]), f"element {i}"
+    for idx, lay in ((0, layouts[0]), (1, layouts[1]), (n_el - 1, last)):
+        sub_w = W.custom(f"max_el_{idx}", [lay], seed=21)
+        L = sub_w.total_tokens
+        t_el = {n: (one[n][:L] if n in ("q", "k", "v") else one[n]) for n in one}
+        _check_sampled(sub_w, t_el, out[idx * per: idx * per + L], seed=idx)
 
 
 def test_empty_batch_is_a_no_op(hgx):
@@ -387,3 +432,78 @@ def test_bounded_wait_reports_timeout_and_context_survives(hgx):
     out, _ = _run(hgx, w, d)
     ref, _, _ = _oracle_full(w, t)
     _compare(out.float().cpu().numpy(), ref, "after-timeout")
+
+
+@pytest.mark.parametrize("poison", ["nan_in_element_1", "inf_in_element_2"])
+def test_non_finite_v_of_a_later_element_does_not_leak(hgx, poison):
+    """A key block that runs past the end of its batch element also covers the next
+    element's first keys. Their probabilities are exact zeros, but 0 * NaN = NaN, so the
+    kernel must not let those V rows into the earlier element's P V: with NaN (or inf) V in
+    a later element, every earlier element still matches the oracle element by element."""
+    H, a = hgx
+    w = W.custom("poison", [[(200, W.CAUSAL), (100, W.FULL_SEQUENCE)], [(90, W.FULL_IN_SEGMENT), (60, W.CAUSAL)],
+                            [(77, W.FULL_SEQUENCE)]], seed=41)
+    cu = W.cu_seqlens(w)  # 0, 300, 450, 527: elements 0 and 1 end inside a 128-key block
+    t = W.tensors(w)
+    v = t["v"].clone()
+    if poison == "nan_in_element_1":
+        v[int(cu[1]):int(cu[1]) + 84] = float("nan")
+        clean = [0]
+    else:
+        v[int(cu[2]):int(cu[3])] = float("inf")
+        clean = [0, 1]
+    t["v"] = v
+    d = {n: x.cuda() for n, x in t.items()}
+    d["pos"] = torch.from_numpy(W.positions(w)).cuda()
+    out, _ = _run(hgx, w, d)
+    ref, _, _ = _oracle_full(w, t)
+    got = out.float().cpu().numpy()
+    for b in clean:
+        r0, r1 = int(cu[b]), int(cu[b + 1])
+        _compare(got[r0:r1], ref[r0:r1], f"{poison}: element {b}")
+
+
+@pytest.mark.parametrize("case", ["c0", "c1", "random_a", "random_b", "reuse"])
+def test_split_items_and_combine_elementwise(hgx, case):
+    """Split work items: with HGX_DEBUG_SPLIT_TEST every prefix-form item of two or more key
+    blocks runs as two halves by key blocks, whose partial (O, row maximum, row sum) the
+    combine kernel merges; element by element against the oracle (the 2048^2 CFG pair and
+    the Hunyuan GCA workload take the split schedule on their own, in the sampled tests)."""
+    H, _ = hgx
+    a = H.Attention()
+    try:
+        a.set_debug(H.HGX_DEBUG_SPLIT_TEST)
+        w = {"c0": W.config(0), "c1": W.config(1), "random_a": W.random_workload(61, max_batch=3, max_len=900),
+             "random_b": W.random_workload(62, max_batch=4, max_len=700, allow_empty=True),
+             "reuse": W.config(1)}[case]
+        if w.total_tokens == 0:
+            pytest.skip("empty draw")
+        t, d = _device_inputs(w)
+        cu, segs, cu_segs = _desc(w)
+        assert H.schedule(cu, segs, cu_segs, 148, 2)[:, 5].max() >= 0  # something is split
+        out = _nan_like(d["q"])
+        if case == "reuse":  # prefix reuse on split items: rows before <|tms|> are kept
+            first = [128, 16]
+            out.fill_(3.0)
+            # the reused rows' k must already hold k': rotate a copy, keep the prefix rows
+            qr, kr = d["q"].clone(), d["k"].clone()
+            a.prologue(qr, kr, d["pos"], d["wq"], d["wk"])
+            prefix = torch.zeros(w.total_tokens, dtype=torch.bool, device="cuda")
+            for b in range(2):
+                prefix[int(cu[b]):int(cu[b]) + first[b]] = True
+            k_in = torch.where(prefix[:, None, None], kr, d["k"])
+            a.forward_from(d["q"], k_in, d["v"], out, d["pos"], d["wq"], d["wk"], cu, segs, cu_segs, first)
+            assert a.sync_status() == H.HGX_OK
+            ref, _, _ = _oracle_full(w, t)
+            got = out.float().cpu().numpy()
+            for b in range(2):
+                r0, r1 = int(cu[b]), int(cu[b + 1])
+                assert (got[r0:r0 + first[b]] == 3.0).all()
+                _compare(got[r0 + first[b]:r1], ref[r0 + first[b]:r1], f"reuse element {b}")
+            return
+        a.forward(d["q"], d["k"], d["v"], out, d["pos"], d["wq"], d["wk"], cu, segs, cu_segs)
+        assert a.sync_status() == H.HGX_OK
+        ref, _, _ = _oracle_full(w, t)
+        _compare(out.float().cpu().numpy(), ref, f"split {w.name}")
+    finally:
+        a.close()

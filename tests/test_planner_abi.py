@@ -232,9 +232,9 @@ def test_set_debug_rejects_unknown_flags():
     with pytest.raises(B.HgxError):
         a.set_debug(0x80)
     a.set_debug(B.HGX_DEBUG_CHECKED, 10_000_000)
-    a.set_debug(B.HGX_DEBUG_FAIL_ALLOC | B.HGX_DEBUG_CHECKED | B.HGX_DEBUG_STALL_TEST)
+    a.set_debug(B.HGX_DEBUG_FAIL_ALLOC | B.HGX_DEBUG_CHECKED | B.HGX_DEBUG_STALL_TEST | B.HGX_DEBUG_SPLIT_TEST)
     with pytest.raises(B.HgxError):
-        a.set_debug(8)
+        a.set_debug(16)
     a.close()
 
 
@@ -333,3 +333,66 @@ def test_binding_rejects_wrong_tensors_before_the_library():
         assert e.value.status == B.HGX_ERR_INVALID_ARG, what
     check(torch.zeros(T + 2, 32, 128, dtype=bf), "bf16", (32, 128), T)  # more rows than needed is fine
     check(torch.zeros(128, dtype=bf), "bf16", (128,), None)
+
+
+def _lpt_makespan(costs, ctas):
+    import heapq
+
+    h = [(0, c) for c in range(min(ctas, len(costs)))]
+    for cost in sorted(costs, reverse=True):
+        load, c = heapq.heappop(h)
+        heapq.heappush(h, (load + cost, c))
+    return max(load for load, _ in h)
+
+
+@pytest.mark.parametrize("case", ["c1", "c2", "c3", "c4", "multigen", "random_a", "random_b", "holes"])
+@pytest.mark.parametrize("split_test", [False, True])
+def test_split_schedule_covers_every_key_block_once(case, split_test):
+    mode = 2 if split_test else 1
+    """The persistent-CTA schedule, with items split by key blocks where that balances the
+    CTAs better: for every (query block, KV head) the key-block ranges of its items
+    partition the unsplit item's range exactly; a split item has exactly two halves with
+    partial slots 2i and 2i + 1 (all slots distinct); list-form (Gen Image hole) items are
+    never split; and the schedule's makespan never exceeds the longest-first assignment's.
+    The 2048^2 CFG pair (1040 equal items on 148 CTAs) must split."""
+    w = {"c1": W.config(1), "c2": W.config(2), "c3": W.config(3), "c4": W.config(4),
+         "multigen": W.CONFIG_BY_NAME["hunyuan_multigen_9088"],
+         "random_a": W.random_workload(31, max_batch=4, max_len=3000),
+         "random_b": W.random_workload(32, max_batch=2, max_len=6000),
+         "holes": W.random_workload(33, max_batch=3, max_len=4000, kinds=(0, 2, 3, 3))}[case]
+    cu, segs, cu_segs = _desc(w)
+    base = B.schedule(cu, segs, cu_segs, 1)  # one CTA: nothing to balance, nothing split
+    assert (base[:, 5] == -1).all() and (base[:, 3] == 0).all()
+    whole = {(int(r[1]), int(r[2])): (int(r[4]), int(r[6]), int(r[7])) for r in base}
+    ctas = 148
+    s = B.schedule(cu, segs, cu_segs, ctas, mode)
+    groups = {}
+    for r in s:
+        groups.setdefault((int(r[1]), int(r[2])), []).append(r)
+    assert set(groups) == set(whole)
+    slots = []
+    for key, rows in groups.items():
+        n, n_full, list_off = whole[key]
+        rows = sorted(rows, key=lambda r: r[3])
+        assert all(int(r[6]) == n_full for r in rows)
+        if len(rows) == 1:
+            assert rows[0][5] == -1 and rows[0][3] == 0 and rows[0][4] == n
+            continue
+        assert len(rows) == 2 and list_off < 0, (key, rows)
+        a, b = rows
+        assert a[3] == 0 and a[4] >= 1 and b[3] == a[4] and b[4] >= 1 and a[4] + b[4] == n
+        assert a[5] % 2 == 0 and b[5] == a[5] + 1
+        slots += [int(a[5]), int(b[5])]
+    assert sorted(slots) == list(range(len(slots)))
+    # execution order: CTAs in order, every CTA's items contiguous
+    assert (np.diff(s[:, 0]) >= 0).all()
+    used = int(s[:, 0].max()) + 1
+    loads = np.bincount(s[:, 0], weights=s[:, 4] + 2, minlength=used)
+    lpt = _lpt_makespan([int(r[4]) + 2 for r in base], ctas)
+    if not split_test:
+        assert loads.max() <= lpt
+    if case == "c2" and not split_test:
+        assert len(slots) > 0 and loads.max() < lpt
+    if split_test:  # the test hook splits every prefix-form item of two or more key blocks
+        for key, (n, _, list_off) in whole.items():
+            assert len(groups[key]) == (2 if list_off < 0 and n >= 2 else 1), key

@@ -21,6 +21,7 @@ from .binding import (  # noqa: F401
     HGX_DEBUG_CHECKED,
     HGX_DEBUG_STALL_TEST,
     HGX_DEBUG_FAIL_ALLOC,
+    HGX_DEBUG_SPLIT_TEST,
     HGX_ROPE_MROPE_INTERLEAVED,
     HGX_ROPE_2D_ALTERNATING,
     HGX_ROPE_2D_HALVES,
@@ -31,5 +32,6 @@ from .binding import (  # noqa: F401
     library_path,
     row_limits,
     visible_pairs,
+    schedule,
     classify,
 )

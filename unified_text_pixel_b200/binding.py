@@ -15,7 +15,7 @@ import numpy as np
 HGX_OK, HGX_ERR_INVALID_ARG, HGX_ERR_UNSUPPORTED, HGX_ERR_OOM, HGX_ERR_CUDA, HGX_ERR_TIMEOUT = range(6)
 HGX_SEG_CAUSAL, HGX_SEG_FULL_SEQUENCE, HGX_SEG_FULL_IN_SEGMENT, HGX_SEG_GEN_IMAGE = 0, 1, 2, 3
 HGX_TILE_SKIP, HGX_TILE_PARTIAL, HGX_TILE_FULL = 0, 1, 2
-HGX_DEBUG_CHECKED, HGX_DEBUG_STALL_TEST, HGX_DEBUG_FAIL_ALLOC = 1, 2, 4
+HGX_DEBUG_CHECKED, HGX_DEBUG_STALL_TEST, HGX_DEBUG_FAIL_ALLOC, HGX_DEBUG_SPLIT_TEST = 1, 2, 4, 8
 HGX_ROPE_MROPE_INTERLEAVED, HGX_ROPE_2D_ALTERNATING, HGX_ROPE_2D_HALVES = 0, 1, 2
 
 _STATUS = {0: "HGX_OK", 1: "HGX_ERR_INVALID_ARG", 2: "HGX_ERR_UNSUPPORTED", 3: "HGX_ERR_OOM",
@@ -60,6 +60,8 @@ _SIGS = {
     "hgx_attn_row_limits": (ctypes.c_int, [ctypes.c_int32] + [ctypes.c_void_p] * 4 + [ctypes.c_size_t]),
     "hgx_attn_classify": (ctypes.c_int, [ctypes.c_int32] + [ctypes.c_void_p] * 6 + [ctypes.c_size_t, ctypes.c_void_p]),
     "hgx_attn_visible_pairs": (ctypes.c_int, [ctypes.c_int32] + [ctypes.c_void_p] * 4),
+    "hgx_attn_schedule": (ctypes.c_int, [ctypes.c_int32] + [ctypes.c_void_p] * 3 + [ctypes.c_int32, ctypes.c_int32,
+                          ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "hgx_attn_sync_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     "hgx_attn_set_debug": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_uint32, ctypes.c_uint64]),
 }
@@ -104,6 +106,25 @@ def row_limits(cu_seqlens, segs, cu_segs) -> np.ndarray:
     st = lib().hgx_attn_row_limits(len(cu) - 1, _ptr(cu), _ptr(sg), _ptr(cs), _ptr(out), T)
     if st != HGX_OK:
         raise HgxError(st, "hgx_attn_row_limits")
+    return out
+
+
+def schedule(cu_seqlens, segs, cu_segs, ctas: int, mode: int = 0) -> np.ndarray:
+    """The attention kernel's persistent-CTA schedule: int32 [items, 8] rows of
+    (cta, q0, kv_head, kb0, n_total, part, n_full, list_off) in execution order. mode 0: the
+    library's policy; 1: split items whenever that balances better; 2: split every item."""
+    cu, sg, cs = _descriptor(cu_seqlens, segs, cu_segs)
+    n = ctypes.c_size_t()
+    L = lib()
+    st = L.hgx_attn_schedule(len(cu) - 1, _ptr(cu), _ptr(sg), _ptr(cs), int(ctas), int(mode), None, 0,
+                             ctypes.byref(n))
+    if st != HGX_OK:
+        raise HgxError(st, "hgx_attn_schedule")
+    out = np.zeros((n.value, 8), dtype=np.int32)
+    st = L.hgx_attn_schedule(len(cu) - 1, _ptr(cu), _ptr(sg), _ptr(cs), int(ctas), int(mode), _ptr(out),
+                             n.value, ctypes.byref(n))
+    if st != HGX_OK:
+        raise HgxError(st, "hgx_attn_schedule")
     return out
 
 

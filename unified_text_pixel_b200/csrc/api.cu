@@ -31,6 +31,7 @@ struct hgx_attn_handle {
   std::vector<int32_t> key_cu, key_cu_segs;
   std::vector<hgx_segment> key_segs;
   std::vector<int32_t> key_first;  // first recomputed row per element; empty = all rows
+  bool key_split_test = false;     // planned under HGX_DEBUG_SPLIT_TEST
   hgx::Plan plan;
   int plan_device = -1;
 
@@ -50,6 +51,12 @@ struct hgx_attn_handle {
   size_t hole_masks_cap = 0;
   int32_t* d_cta_offsets = nullptr;  // the persistent CTAs' item lists
   size_t cta_offsets_cap = 0;
+  // split items: their list for the combine kernel and the partial results (fp32 O, then
+  // (M, l) pairs), sized for the largest plan so far
+  hgx::WorkItem* d_splits = nullptr;
+  size_t splits_cap = 0;
+  void* d_partial = nullptr;
+  size_t partial_cap = 0;
   // (cos, sin) per (token, frequency) for the QKV projection's epilogue
   void* d_rope_cs = nullptr;
   size_t rope_cs_cap = 0;
@@ -61,6 +68,13 @@ struct hgx_attn_handle {
 };
 
 namespace {
+
+#ifndef HGX_SPLIT_KV
+#define HGX_SPLIT_KV 0
+#endif
+// 1: the planner may split items by key blocks when that balances the persistent CTAs
+// better (hgx::assign_ctas); 0: longest-processing-time assignment only
+constexpr bool kSplitKV = HGX_SPLIT_KV != 0;
 
 using PFN_encodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                      const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -148,6 +162,7 @@ hgx_status ensure_device(hgx_attn_handle* h) {
 bool same_descriptor(const hgx_attn_handle* h, int32_t batch, const int32_t* cu,
                      const hgx_segment* segs, const int32_t* cu_segs, const int32_t* first) {
   if (h->key_batch != batch) return false;
+  if (h->key_split_test != ((h->flags & HGX_DEBUG_SPLIT_TEST) != 0)) return false;
   if (first ? (h->key_first.size() != static_cast<size_t>(batch) ||
                std::memcmp(h->key_first.data(), first, sizeof(int32_t) * batch) != 0)
             : !h->key_first.empty())
@@ -172,9 +187,11 @@ hgx_status prepare_plan(hgx_attn_handle* h, cudaStream_t stream, int32_t batch,
     hgx_status st =
         hgx::build_plan(batch, cu, segs, cu_segs, h->cfg.num_kv_heads, &plan, &err, first);
     if (st != HGX_OK) return fail(h, st, err);
-    hgx::assign_ctas(&plan, h->num_sms);
+    const bool split_test = (h->flags & HGX_DEBUG_SPLIT_TEST) != 0;
+    hgx::assign_ctas(&plan, h->num_sms, kSplitKV, split_test);
     h->plan = std::move(plan);
     h->key_batch = batch;
+    h->key_split_test = split_test;
     h->key_cu.assign(cu, cu + batch + 1);
     h->key_cu_segs.assign(cu_segs, cu_segs + batch + 1);
     h->key_segs.assign(segs, segs + cu_segs[batch]);
@@ -204,6 +221,8 @@ hgx_status prepare_plan(hgx_attn_handle* h, cudaStream_t stream, int32_t batch,
        pl.hole_masks.size() * sizeof(uint32_t)},
       {reinterpret_cast<void**>(&h->d_cta_offsets), &h->cta_offsets_cap, pl.cta_offsets.data(),
        pl.cta_offsets.size() * sizeof(int32_t)},
+      {reinterpret_cast<void**>(&h->d_splits), &h->splits_cap, pl.splits.data(),
+       pl.splits.size() * sizeof(hgx::WorkItem)},
   };
   size_t need = 0;
   for (const Upload& u : up) {
@@ -220,6 +239,22 @@ hgx_status prepare_plan(hgx_attn_handle* h, cudaStream_t stream, int32_t batch,
       *u.cap = u.bytes;
     }
     need += (u.bytes + 255) & ~size_t(255);
+  }
+  // partial results of split items (written and read on the device only)
+  const size_t slots = 2 * pl.splits.size();
+  const size_t partial_bytes =
+      slots * (hgx::kPartialSlotFloats * sizeof(float) + hgx::kPartialSlotRows * sizeof(float2));
+  if (partial_bytes > h->partial_cap) {
+    if (h->flags & HGX_DEBUG_FAIL_ALLOC) {
+      h->flags &= ~HGX_DEBUG_FAIL_ALLOC;
+      return fail(h, HGX_ERR_OOM, "cudaMalloc of the partial results failed (injected)");
+    }
+    if (h->d_partial) cudaFree(h->d_partial);
+    h->d_partial = nullptr;
+    h->partial_cap = 0;
+    if (cudaMalloc(&h->d_partial, partial_bytes) != cudaSuccess)
+      return fail(h, HGX_ERR_OOM, "cudaMalloc of the partial results failed");
+    h->partial_cap = partial_bytes;
   }
   cudaError_t e;
   // the previous upload may still be reading the staging buffer
@@ -282,12 +317,22 @@ hgx_status run_attention(hgx_attn_handle* h, cudaStream_t stream, const void* q,
   p.hole_base = h->plan.has_holes ? h->d_hole_base : nullptr;
   p.hole_masks = h->plan.has_holes ? h->d_hole_masks : nullptr;
   p.out = out;
+  const size_t slots = 2 * h->plan.splits.size();
+  p.partial_o = slots ? static_cast<float*>(h->d_partial) : nullptr;
+  p.partial_ml = slots ? reinterpret_cast<float2*>(static_cast<float*>(h->d_partial) +
+                                                   slots * hgx::kPartialSlotFloats)
+                       : nullptr;
   p.scale_log2 = h->scale * 1.4426950408889634f;
   p.flags = h->flags;
   p.err = h->d_err;
   p.wait_limit_ns = h->wait_limit_ns;
   cudaError_t e = hgx::launch_attention(stream, mq, mk, mv, p, h->plan.grid);
   if (e != cudaSuccess) return cuda_fail(h, e, "attention launch");
+  if (slots) {
+    e = hgx::launch_combine(stream, h->d_splits, static_cast<int32_t>(h->plan.splits.size()), p.partial_o,
+                            p.partial_ml, out);
+    if (e != cudaSuccess) return cuda_fail(h, e, "combine launch");
+  }
   return HGX_OK;
 }
 
@@ -412,6 +457,8 @@ void hgx_attn_destroy(hgx_attn_handle* h) {
   if (h->d_hole_base) cudaFree(h->d_hole_base);
   if (h->d_hole_masks) cudaFree(h->d_hole_masks);
   if (h->d_cta_offsets) cudaFree(h->d_cta_offsets);
+  if (h->d_splits) cudaFree(h->d_splits);
+  if (h->d_partial) cudaFree(h->d_partial);
   if (h->d_rope_cs) cudaFree(h->d_rope_cs);
   if (h->d_err) cudaFree(h->d_err);
   if (h->h_stage) cudaFreeHost(h->h_stage);
@@ -619,6 +666,36 @@ hgx_status hgx_attn_classify(int32_t batch, const int32_t* cu_seqlens_host,
   return HGX_OK;
 }
 
+hgx_status hgx_attn_schedule(int32_t batch, const int32_t* cu_seqlens_host,
+                             const hgx_segment* segs_host, const int32_t* cu_segs_host, int32_t ctas,
+                             int32_t mode, int32_t* out, size_t cap, size_t* n_items) {
+  if (n_items) *n_items = 0;
+  if (ctas < 1 || mode < 0 || mode > 2) return HGX_ERR_INVALID_ARG;
+  hgx::Plan plan;
+  std::string err;
+  hgx_status st = hgx::build_plan(batch, cu_seqlens_host, segs_host, cu_segs_host, 8, &plan, &err);
+  if (st != HGX_OK) return st;
+  hgx::assign_ctas(&plan, ctas, mode == 0 ? kSplitKV : true, mode == 2);
+  const size_t n = plan.items.size();
+  if (n_items) *n_items = n;
+  if (!out) return HGX_OK;
+  if (cap < n) return HGX_ERR_INVALID_ARG;
+  for (int32_t c = 0; c < plan.grid; ++c)
+    for (int32_t i = plan.cta_offsets[static_cast<size_t>(c)]; i < plan.cta_offsets[static_cast<size_t>(c) + 1]; ++i) {
+      const hgx::WorkItem& it = plan.items[static_cast<size_t>(i)];
+      int32_t* r = out + 8 * static_cast<size_t>(i);
+      r[0] = c;
+      r[1] = it.q0;
+      r[2] = it.g;
+      r[3] = it.kb0;
+      r[4] = it.n_total;
+      r[5] = it.part;
+      r[6] = it.n_full;
+      r[7] = it.list_off;
+    }
+  return HGX_OK;
+}
+
 hgx_status hgx_attn_visible_pairs(int32_t batch, const int32_t* cu_seqlens_host,
                                   const hgx_segment* segs_host, const int32_t* cu_segs_host,
                                   uint64_t* pairs) {
@@ -653,7 +730,7 @@ hgx_status hgx_attn_sync_status(hgx_attn_handle* h, void* stream) {
 
 hgx_status hgx_attn_set_debug(hgx_attn_handle* h, uint32_t flags, uint64_t wait_limit_ns) {
   if (!h) return HGX_ERR_INVALID_ARG;
-  if (flags & ~(HGX_DEBUG_CHECKED | HGX_DEBUG_STALL_TEST | HGX_DEBUG_FAIL_ALLOC))
+  if (flags & ~(HGX_DEBUG_CHECKED | HGX_DEBUG_STALL_TEST | HGX_DEBUG_FAIL_ALLOC | HGX_DEBUG_SPLIT_TEST))
     return fail(h, HGX_ERR_INVALID_ARG, "unknown debug flag");
   h->flags = flags;
   h->wait_limit_ns = wait_limit_ns ? wait_limit_ns : 2000000000ull;

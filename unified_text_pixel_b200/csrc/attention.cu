@@ -66,8 +66,15 @@ constexpr int kThreads = 128 + 2 * kSoftmaxThreads;
 // register budgets after setmaxnreg (launch: 384 x 168 or 640 x 96 registers)
 constexpr uint32_t kRegsLow = kSplit == 1 ? 120 : 64;   // producer/MMA warpgroup
 constexpr uint32_t kRegsHigh = kSplit == 1 ? 192 : 104;  // softmax warpgroups
+#ifndef HGX_Q_BUFS
+#define HGX_Q_BUFS 1
+#endif
+// Q buffers (each both Q tiles of an item): 2 loads the next item's Q during the current
+// item, which leaves room for 3 K/V slots only
+constexpr int kQBufs = HGX_Q_BUFS;
+static_assert(kQBufs == 1 || kQBufs == 2, "Q buffers");
 #ifndef HGX_KV_STAGES
-#define HGX_KV_STAGES 4
+#define HGX_KV_STAGES (HGX_Q_BUFS == 2 ? 3 : 4)
 #endif
 constexpr int kStages = HGX_KV_STAGES;        // K/V ring slots
 #ifndef HGX_P_PARTS
@@ -77,16 +84,22 @@ constexpr int kStages = HGX_KV_STAGES;        // K/V ring slots
 // that the PV MMAs of the first parts overlap the exponentials of the later ones
 constexpr int kPParts = HGX_P_PARTS;
 static_assert(kPParts == 1 || kPParts == 2 || kPParts == 4, "P parts");
+#ifndef HGX_EPI_LOAD_ALL
+#define HGX_EPI_LOAD_ALL 0
+#endif
+// 1: the epilogue loads the whole O row from tensor memory with one wait and releases O to
+// the next item's PV before it stores (instead of four load-wait-store rounds)
+constexpr bool kEpiLoadAll = HGX_EPI_LOAD_ALL != 0;
 constexpr uint32_t kTileBytes = 32768;        // 128 rows x 128 bf16
 constexpr uint32_t kHalfBytes = 16384;        // 128 rows x 64 bf16 (one 128-byte swizzle span)
 constexpr uint32_t kQBytes = 2 * kTileBytes;  // both Q tiles of an item
-constexpr uint32_t kRingOffset = kQBytes;
+constexpr uint32_t kRingOffset = kQBufs * kQBytes;
 constexpr uint32_t kBarOffset = kRingOffset + kStages * kTileBytes;
 // barrier slots (8 bytes each)
 enum : uint32_t {
-  BAR_Q_FULL = 0,
-  BAR_Q_EMPTY = 1,
-  BAR_KV_FULL = 2,                   // + slot
+  BAR_Q_FULL = 0,                    // + Q buffer
+  BAR_Q_EMPTY = BAR_Q_FULL + kQBufs, // + Q buffer
+  BAR_KV_FULL = BAR_Q_EMPTY + kQBufs,  // + slot
   BAR_KV_EMPTY = BAR_KV_FULL + kStages,
   BAR_S_FULL = BAR_KV_EMPTY + kStages,  // + tile
   BAR_PA_FULL = BAR_S_FULL + 2,         // + tile * (kPParts - 1) + part: that part of P written
@@ -104,6 +117,7 @@ constexpr uint32_t kXchgOffset = kMiscOffset + 16;
 constexpr uint32_t kXchgBytes = kSplit == 2 ? 2 * 2 * 2 * 128 * 4 : 0;
 constexpr uint32_t kSmemUsed = kXchgOffset + kXchgBytes;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // slack to align the base to 1024 B
+static_assert(kSmemBytes <= 232448, "more dynamic shared memory than an sm_100 CTA may have");
 
 constexpr uint32_t kTmemCols = 512;
 __host__ __device__ constexpr uint32_t col_s(int x) { return 128u * x; }        // S0, S1
@@ -215,8 +229,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   Ctx c{base + kBarOffset, abort_flag, p.err, p.wait_limit_ns};
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_addr(c, BAR_Q_FULL), 1);
-    mbar_init(bar_addr(c, BAR_Q_EMPTY), 1);
+    for (int b = 0; b < kQBufs; ++b) {
+      mbar_init(bar_addr(c, BAR_Q_FULL + b), 1);
+      mbar_init(bar_addr(c, BAR_Q_EMPTY + b), 1);
+    }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(bar_addr(c, BAR_KV_FULL + s), 1);
       mbar_init(bar_addr(c, BAR_KV_EMPTY + s), 1);
@@ -261,23 +277,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tmap_q);
         tma_prefetch_desc(&tmap_k);
         tma_prefetch_desc(&tmap_v);
-        uint32_t pos = 0, qe_par = 0, q_loads = 0;
+        uint32_t pos = 0, q_loads = 0;
         uint32_t loaded = 0, last_par = 0;  // per slot: ever loaded, parity of its last load
         bool ok = true;
         for (int w = first_item(p); ok && w < end_item(p); w = next_item(p, w)) {
           const WorkItem it = p.items[w];
-          if (q_loads > 0) {
-            ok = wait_bounded(c, bar_addr(c, BAR_Q_EMPTY), qe_par, SITE_PRODUCER);
-            qe_par ^= 1u;
+          const uint32_t qb = q_loads % kQBufs;  // Q buffer of this item
+          if (q_loads >= static_cast<uint32_t>(kQBufs)) {
+            ok = wait_bounded(c, bar_addr(c, BAR_Q_EMPTY + qb), ((q_loads / kQBufs) - 1) & 1u, SITE_PRODUCER);
             if (!ok) break;
           }
-          mbar_arrive_expect_tx(bar_addr(c, BAR_Q_FULL), kQBytes);
+          mbar_arrive_expect_tx(bar_addr(c, BAR_Q_FULL + qb), kQBytes);
           for (int x = 0; x < 2; ++x) {
             // a tile that starts past the last token only holds rows that are never stored:
             // start it at the last token so that no box lies wholly outside the tensor
             const int32_t t0 = min(it.q0 + 32 * x, p.total_tokens - 1);
             for (int hf = 0; hf < 2; ++hf)
-              tma_load_3d(sQ + x * kTileBytes + hf * kHalfBytes, &tmap_q, bar_addr(c, BAR_Q_FULL),
+              tma_load_3d(sQ + qb * kQBytes + x * kTileBytes + hf * kHalfBytes, &tmap_q, bar_addr(c, BAR_Q_FULL + qb),
                           64 * hf, 4 * it.g, t0);
           }
           ++q_loads;
@@ -292,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               mbar_arrive_expect_tx(full, kTileBytes);
               const CUtensorMap* map = kv == 0 ? &tmap_k : &tmap_v;
               const int32_t kb =
-                it.list_off < 0 ? j : static_cast<int32_t>(p.kblocks[it.list_off + j] & kListBlockMask);
+                it.list_off < 0 ? it.kb0 + j : static_cast<int32_t>(p.kblocks[it.list_off + j] & kListBlockMask);
             for (int hf = 0; hf < 2; ++hf)
                 tma_load_3d(sRing + slot * kTileBytes + hf * kHalfBytes, map, full, 64 * hf, it.g,
                             it.kv0 + 128 * kb);
@@ -306,13 +322,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         // path they all have, and these waits return at once)
         for (int s = 0; s < kStages; ++s)
           if (loaded & (1u << s)) wait_drain(c, bar_addr(c, BAR_KV_FULL + s), (last_par >> s) & 1u, SITE_DRAIN);
-        if (q_loads > 0) wait_drain(c, bar_addr(c, BAR_Q_FULL), (q_loads - 1) & 1u, SITE_DRAIN);
+        for (uint32_t b = 0; b < static_cast<uint32_t>(kQBufs) && b < q_loads; ++b) {  // last load of buffer b
+          const uint32_t last = q_loads - 1 - ((q_loads - 1 - b) % kQBufs);
+          wait_drain(c, bar_addr(c, BAR_Q_FULL + b), (last / kQBufs) & 1u, SITE_DRAIN);
+        }
       }
       __syncwarp();
     } else if (warp == 1) {
       // ------------------------------------------------------------------ MMA issuer
       if (lane == 0) {
-        uint32_t pos = 0, qf_par = 0;
+        uint32_t pos = 0, q_items = 0;
         uint32_t pa_par[2] = {0, 0}, p_par[2] = {0, 0}, oe_par[2] = {0, 0};  // pa: all parts share it
         bool first = true, ok = true;
         auto wait_kv = [&](uint32_t ps) {
@@ -320,8 +339,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                               SITE_MMA);
         };
         // descriptors of both Q tiles and of K / V in ring slot 0 (slot s: + s * 32 KB >> 4)
-        const uint64_t dq0 = smem_desc_sw128(sQ, 16, 1024);
-        const uint64_t dq1 = smem_desc_sw128(sQ + kTileBytes, 16, 1024);
+        const uint64_t dq0_base = smem_desc_sw128(sQ, 16, 1024);
+        const uint64_t dq1_base = smem_desc_sw128(sQ + kTileBytes, 16, 1024);
         const uint64_t dk0 = smem_desc_sw128(sRing, 16, 1024);
         const uint64_t dv0 = smem_desc_sw128(sRing, kHalfBytes, 1024);
         auto kdesc = [&](uint32_t ps) { return dk0 + (ps % kStages) * (kTileBytes >> 4); };
@@ -365,8 +384,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int w = first_item(p); ok && w < end_item(p); w = next_item(p, w)) {
           const WorkItem it = p.items[w];
           const int n = it.n_total;
-          if (!(ok = wait_bounded(c, bar_addr(c, BAR_Q_FULL), qf_par, SITE_MMA))) break;
-          qf_par ^= 1u;
+          const uint32_t qb = q_items % kQBufs;
+          if (!(ok = wait_bounded(c, bar_addr(c, BAR_Q_FULL + qb), (q_items / kQBufs) & 1u, SITE_MMA))) break;
+          ++q_items;
+          const uint64_t dq0 = dq0_base + qb * (kQBytes >> 4), dq1 = dq1_base + qb * (kQBytes >> 4);
           uint32_t kpos = pos++;
           if (!(ok = wait_kv(kpos))) break;
           tc_fence_after();
@@ -374,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(bar_addr(c, BAR_S_FULL + 0));
           issue_qk(tmem + col_s(1), dq1, kdesc(kpos));
           mma_commit(bar_addr(c, BAR_S_FULL + 1));
-          if (n == 1) mma_commit(bar_addr(c, BAR_Q_EMPTY));
+          if (n == 1) mma_commit(bar_addr(c, BAR_Q_EMPTY + qb));
           release(kpos);
           for (int j = 1; j < n; ++j) {
             const uint32_t vpos = pos++;
@@ -387,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             release(vpos);
             issue_qk(tmem + col_s(1), dq1, kdesc(kpos));
             mma_commit(bar_addr(c, BAR_S_FULL + 1));
-            if (j == n - 1) mma_commit(bar_addr(c, BAR_Q_EMPTY));
+            if (j == n - 1) mma_commit(bar_addr(c, BAR_Q_EMPTY + qb));
             release(kpos);
           }
           if (!ok) break;
@@ -428,6 +449,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sl2 = p.scale_log2;
     uint32_t s_par = 0, o_par = 0;
     int xpar = 0;  // exchange buffer parity
+    uint32_t ring = 0;        // K/V ring position of the next key block's K (V follows it)
+    uint8_t* const ring_g = gbase + kRingOffset;
     // one decision for every thread of the tile: its two halves must leave together
     auto agree = [&](bool v) {
       if constexpr (kSplit == 1) return __all_sync(0xffffffffu, v);
@@ -448,12 +471,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < it.n_total; ++j) {
         // key block and its class (read before the wait, which hides the load)
         const uint32_t entry = listed ? p.kblocks[it.list_off + j] : 0u;
-        const int32_t kb = listed ? static_cast<int32_t>(entry & kListBlockMask) : j;
-        const bool full = listed ? (entry >> kListClassShift) == HGX_TILE_FULL : j < it.n_full;
+        const int32_t kb = listed ? static_cast<int32_t>(entry & kListBlockMask) : it.kb0 + j;
+        const bool full = listed ? (entry >> kListClassShift) == HGX_TILE_FULL : kb < it.n_full;
         uint4 hm = make_uint4(0u, 0u, 0u, 0u);
         if (!full && hbase >= 0)
           hm = *reinterpret_cast<const uint4*>(p.hole_masks + 4 * static_cast<size_t>(hbase + kb));
         bool got = wait_bounded(c, bar_addr(c, BAR_S_FULL + x), s_par, SITE_SOFTMAX);
+        const uint32_t vpos = ring + 1;
+        ring += 2;
+        // A key block that runs past the end of its batch element into the next one: the
+        // probabilities of those keys are exact zeros, but their V rows belong to the next
+        // element and 0 * inf or 0 * NaN would be NaN, so tile 0 zeroes them in shared
+        // memory once the V tile has landed and before it publishes any P of this block
+        // (the PV MMAs of both tiles read V after that). Blocks past the last token read
+        // zeros from the tensor map already.
+        if (x == 0 && 128 * kb + 128 > it.len && it.kv0 + it.len < p.total_tokens) {
+          got = got && wait_bounded(c, bar_addr(c, BAR_KV_FULL + vpos % kStages), (vpos / kStages) & 1u,
+                                    SITE_SOFTMAX);
+          if (half == 0 && row >= it.len - 128 * kb) {
+            uint8_t* v_row = ring_g + (vpos % kStages) * kTileBytes + row * 128;
+            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+              for (int e = 0; e < 8; ++e) reinterpret_cast<uint4*>(v_row + hf * kHalfBytes)[e] = z;
+          }
+          fence_proxy_async_smem();  // the tensor core reads these rows through the async proxy
+        }
         if constexpr (kSplit == 1) {
           if (!(ok = __all_sync(0xffffffffu, got))) break;
         }
@@ -612,9 +656,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       o_par ^= 1u;
       tc_fence_after();
+      if (it.part >= 0) {
+        // one part of a split item: unnormalised O, the exponent shift and the row sum, for
+        // the combine kernel (a row that saw no key of this part has l = 0 and M = -inf)
+        const size_t prow = (static_cast<size_t>(it.part) * 2 + x) * 128 + row;
+        float* po = p.partial_o + prow * 128 + kCols * half;
+#pragma unroll
+        for (int ch = 0; ch < kCols / 32; ++ch) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * ch, o);
+          tmem_wait_ld();
+          if (valid) {
+            float4* d4 = reinterpret_cast<float4*>(po + 32 * ch);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              d4[e] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
+                                  __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
+          }
+        }
+        if (valid && half == 0)
+          p.partial_ml[prow] = make_float2(m_used == -INFINITY ? -INFINITY : m_used * sl2, l);
+        tc_fence_before();
+        mbar_arrive(bar_addr(c, BAR_O_EMPTY + x));
+        continue;
+      }
       const float inv_l = 1.0f / l;
       __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) +
                            (static_cast<size_t>(tok) * 32 + head) * 128 + kCols * half;
+      if constexpr (kEpiLoadAll) {
+        // every tensor-memory load of the row first, one wait, then the stores
+        uint32_t o[kCols / 32][32];
+#pragma unroll
+        for (int ch = 0; ch < kCols / 32; ++ch) tmem_ld32(tO + 32 * ch, o[ch]);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar_addr(c, BAR_O_EMPTY + x));  // O is in registers: the next PV may start
+        if (valid) {
+#pragma unroll
+          for (int ch = 0; ch < kCols / 32; ++ch) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * ch);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              d4[e] = make_uint4(
+                  pack_bf16x2(__uint_as_float(o[ch][8 * e]) * inv_l, __uint_as_float(o[ch][8 * e + 1]) * inv_l),
+                  pack_bf16x2(__uint_as_float(o[ch][8 * e + 2]) * inv_l, __uint_as_float(o[ch][8 * e + 3]) * inv_l),
+                  pack_bf16x2(__uint_as_float(o[ch][8 * e + 4]) * inv_l, __uint_as_float(o[ch][8 * e + 5]) * inv_l),
+                  pack_bf16x2(__uint_as_float(o[ch][8 * e + 6]) * inv_l, __uint_as_float(o[ch][8 * e + 7]) * inv_l));
+          }
+        }
+        continue;
+      }
 #pragma unroll
       for (int ch = 0; ch < kCols / 32; ++ch) {
         uint32_t o[32];
@@ -640,7 +731,42 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// One warp per row of a split item: lane i merges features 4i .. 4i + 3.
+__global__ void __launch_bounds__(256) combine_kernel(const WorkItem* __restrict__ splits, int32_t n_splits,
+                                                      const float* __restrict__ po,
+                                                      const float2* __restrict__ pml, __nv_bfloat16* out) {
+  const int32_t gw = static_cast<int32_t>(blockIdx.x) * 8 + static_cast<int32_t>(threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (gw >= n_splits * 256) return;
+  const WorkItem it = splits[gw >> 8];
+  const int x = (gw >> 7) & 1, row = gw & 127;
+  const int32_t tok = it.q0 + 32 * x + (row >> 2);
+  if (!(tok - it.kv0 < it.len && tok - it.kv0 >= it.first)) return;
+  const size_t ra = (static_cast<size_t>(it.part) * 2 + x) * 128 + row;
+  const size_t rb = ra + kPartialSlotRows;  // slot part + 1
+  const float2 a = pml[ra], b = pml[rb];
+  const float m = fmaxf(a.x, b.x);  // finite: every written row sees at least itself
+  const float wa = a.y > 0.f ? exp2f(a.x - m) : 0.f;
+  const float wb = b.y > 0.f ? exp2f(b.x - m) : 0.f;
+  const float inv = 1.f / (a.y * wa + b.y * wb);
+  const float4 oa = reinterpret_cast<const float4*>(po + ra * 128)[lane];
+  const float4 ob = reinterpret_cast<const float4*>(po + rb * 128)[lane];
+  const uint32_t lo = pack_bf16x2((oa.x * wa + ob.x * wb) * inv, (oa.y * wa + ob.y * wb) * inv);
+  const uint32_t hi = pack_bf16x2((oa.z * wa + ob.z * wb) * inv, (oa.w * wa + ob.w * wb) * inv);
+  const int32_t head = 4 * it.g + (row & 3);
+  reinterpret_cast<uint2*>(out + (static_cast<size_t>(tok) * 32 + head) * 128)[lane] = make_uint2(lo, hi);
+}
+
 }  // namespace
+
+cudaError_t launch_combine(cudaStream_t stream, const WorkItem* splits, int32_t n_splits,
+                           const float* partial_o, const float2* partial_ml, void* out) {
+  if (n_splits <= 0) return cudaSuccess;
+  const int blocks = (n_splits * 256 + 7) / 8;
+  combine_kernel<<<blocks, 256, 0, stream>>>(splits, n_splits, partial_o, partial_ml,
+                                             static_cast<__nv_bfloat16*>(out));
+  return cudaGetLastError();
+}
 
 size_t attention_smem_bytes() { return kSmemBytes; }
 

@@ -33,11 +33,20 @@ struct AttnParams {
   const int32_t* hole_base;    // [T] row's first hole-mask index, -1 = none (holes only)
   const uint32_t* hole_masks;  // 4 words per (segment, key block): hidden keys (holes only)
   void* out;               // bf16 [T, 32, 128]
+  float* partial_o;        // split items: unnormalised O per slot, fp32 [slots][2][128][128]
+  float2* partial_ml;      // split items: (row maximum x scale log2 e, row sum) [slots][2][128]
   float scale_log2;        // softmax scale * log2(e)
   uint32_t flags;          // HGX_DEBUG_* bits
   uint32_t* err;           // device error word (sticky until read)
   uint64_t wait_limit_ns;  // bound of every wait
 };
+
+// Merges the two partial results of every split item into out (bf16):
+// out = (O_a 2^(M_a - M) + O_b 2^(M_b - M)) / (l_a 2^(M_a - M) + l_b 2^(M_b - M)), M = max.
+cudaError_t launch_combine(cudaStream_t stream, const WorkItem* splits, int32_t n_splits,
+                           const float* partial_o, const float2* partial_ml, void* out);
+constexpr size_t kPartialSlotFloats = 2 * 128 * 128;  // fp32 O of one slot
+constexpr size_t kPartialSlotRows = 2 * 128;          // rows (and (M, l) pairs) of one slot
 
 // Bytes of dynamic shared memory the attention kernel needs.
 size_t attention_smem_bytes();

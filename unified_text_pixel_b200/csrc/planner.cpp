@@ -263,28 +263,133 @@ hgx_status build_plan(int32_t batch, const int32_t* cu_seqlens, const hgx_segmen
   return HGX_OK;
 }
 
-void assign_ctas(Plan* plan, int32_t ctas) {
+namespace {
+
+int64_t item_cost(const WorkItem& it) { return it.n_total + kItemOverhead; }
+
+// Longest processing time first; items are sorted longest first. Returns the owner of
+// every item and the makespan.
+int64_t lpt(const std::vector<WorkItem>& items, int32_t g, std::vector<int32_t>* owner) {
+  using Load = std::pair<int64_t, int32_t>;  // (load, cta)
+  std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+  for (int32_t c = 0; c < g; ++c) heap.push({0, c});
+  owner->assign(items.size(), 0);
+  int64_t makespan = 0;
+  for (size_t i = 0; i < items.size(); ++i) {
+    Load l = heap.top();
+    heap.pop();
+    (*owner)[i] = l.second;
+    l.first += item_cost(items[i]);
+    makespan = std::max(makespan, l.first);
+    heap.push(l);
+  }
+  return makespan;
+}
+
+// Wrap-around fill (McNaughton) up to the bound B = ceil((total cost + the overhead of up
+// to g - 1 splits) / g). Produces the items in CTA order, the offsets, the splits and the
+// makespan.
+int64_t wrap_around(const std::vector<WorkItem>& items, int32_t g, std::vector<WorkItem>* out,
+                    std::vector<int32_t>* offsets, std::vector<WorkItem>* splits) {
+  int64_t total = 0;
+  for (const WorkItem& it : items) total += item_cost(it);
+  const int64_t bound = (total + kItemOverhead * (g - 1) + g - 1) / g;
+  out->clear();
+  splits->clear();
+  offsets->assign(static_cast<size_t>(g) + 1, 0);
+  int32_t c = 0;
+  int64_t load = 0, makespan = 0;
+  auto close_cta = [&]() {
+    makespan = std::max(makespan, load);
+    (*offsets)[static_cast<size_t>(c) + 1] = static_cast<int32_t>(out->size());
+    ++c;
+    load = 0;
+  };
+  for (const WorkItem& it : items) {
+    const int64_t cost = item_cost(it);
+    if (c < g - 1 && load + cost > bound) {
+      const int64_t room = bound - load - kItemOverhead;  // key blocks that still fit
+      if (it.list_off < 0 && it.part < 0 && room >= 1 && it.n_total - room >= 1) {
+        const int32_t a = static_cast<int32_t>(room);
+        const int32_t slot = 2 * static_cast<int32_t>(splits->size());
+        WorkItem whole = it;
+        whole.part = slot;
+        splits->push_back(whole);
+        WorkItem head = it;  // the first key blocks: end of this CTA's list
+        head.n_total = a;
+        head.part = slot;
+        out->push_back(head);
+        load += a + kItemOverhead;
+        close_cta();
+        WorkItem tail = it;  // the rest: start of the next CTA's list
+        tail.kb0 = it.kb0 + a;
+        tail.n_total = it.n_total - a;
+        tail.part = slot + 1;
+        out->push_back(tail);
+        load = item_cost(tail);
+        continue;
+      }
+      if (load > 0) close_cta();
+    }
+    out->push_back(it);
+    load += cost;
+  }
+  while (c < g) close_cta();
+  return makespan;
+}
+
+}  // namespace
+
+void assign_ctas(Plan* plan, int32_t ctas, bool allow_split, bool force_split) {
+  plan->splits.clear();
+  if (force_split) {
+    // test hook: every prefix-form item of two or more key blocks becomes two halves
+    std::vector<WorkItem> halves;
+    for (const WorkItem& it : plan->items) {
+      if (it.list_off >= 0 || it.n_total < 2) {
+        halves.push_back(it);
+        continue;
+      }
+      const int32_t slot = 2 * static_cast<int32_t>(plan->splits.size());
+      WorkItem whole = it;
+      whole.part = slot;
+      plan->splits.push_back(whole);
+      WorkItem head = it, tail = it;
+      head.n_total = it.n_total / 2;
+      head.part = slot;
+      tail.kb0 = it.kb0 + head.n_total;
+      tail.n_total = it.n_total - head.n_total;
+      tail.part = slot + 1;
+      halves.push_back(head);
+      halves.push_back(tail);
+    }
+    std::stable_sort(halves.begin(), halves.end(),
+                     [](const WorkItem& x, const WorkItem& y) { return x.n_total > y.n_total; });
+    plan->items.swap(halves);
+  }
   const int32_t n = static_cast<int32_t>(plan->items.size());
   const int32_t g = std::max(1, std::min(ctas, n));
   plan->grid = n ? g : 0;
   plan->cta_offsets.assign(static_cast<size_t>(g) + 1, 0);
+  plan->makespan = 0;
   if (!n) return;
-  // items are sorted by n_total, longest first; the per-item overhead stands for loading Q
-  // and writing O (about two key blocks of work)
-  constexpr int64_t kItemOverhead = 2;
-  using Load = std::pair<int64_t, int32_t>;  // (load, cta)
-  std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
-  for (int32_t c = 0; c < g; ++c) heap.push({0, c});
-  std::vector<int32_t> owner(static_cast<size_t>(n));
-  std::vector<int32_t> count(static_cast<size_t>(g), 0);
-  for (int32_t i = 0; i < n; ++i) {
-    Load l = heap.top();
-    heap.pop();
-    owner[static_cast<size_t>(i)] = l.second;
-    ++count[static_cast<size_t>(l.second)];
-    l.first += plan->items[static_cast<size_t>(i)].n_total + kItemOverhead;
-    heap.push(l);
+  std::vector<int32_t> owner;
+  const int64_t lpt_span = lpt(plan->items, g, &owner);
+  if (allow_split && !force_split && g > 1) {
+    std::vector<WorkItem> wrapped, splits;
+    std::vector<int32_t> offsets;
+    const int64_t span = wrap_around(plan->items, g, &wrapped, &offsets, &splits);
+    if (!splits.empty() && span + kSplitPenalty < lpt_span) {
+      plan->items.swap(wrapped);
+      plan->cta_offsets.swap(offsets);
+      plan->splits.swap(splits);
+      plan->makespan = span;
+      return;
+    }
   }
+  plan->makespan = lpt_span;
+  std::vector<int32_t> count(static_cast<size_t>(g), 0);
+  for (int32_t i = 0; i < n; ++i) ++count[static_cast<size_t>(owner[static_cast<size_t>(i)])];
   for (int32_t c = 0; c < g; ++c) plan->cta_offsets[static_cast<size_t>(c) + 1] = plan->cta_offsets[static_cast<size_t>(c)] + count[static_cast<size_t>(c)];
   std::vector<WorkItem> ordered(static_cast<size_t>(n));
   std::vector<int32_t> at(plan->cta_offsets.begin(), plan->cta_offsets.end() - 1);

@@ -24,11 +24,16 @@ constexpr int32_t kMaxTokens = (1 << 19) - 1;
 // One unit of attention work: one KV head g and its 4 query heads over kBlockTokens
 // consecutive query tokens of one batch element. Layout shared with the kernel.
 //
-// Prefix form (list_off < 0): the item processes key blocks 0 .. n_total-1; blocks
-// [0, n_full) are visible to every row (no mask compare), the rest need the per-row compare.
-// List form (list_off >= 0, items whose rows see a Gen Image hole): the item processes the
-// n_total key blocks listed at kblocks[list_off ...], each entry kb | class << 24 with class
-// an hgx_tile_class (FULL or PARTIAL; skipped blocks are not listed).
+// Prefix form (list_off < 0): the item processes key blocks kb0 .. kb0 + n_total - 1; blocks
+// below n_full are visible to every row (no mask compare), the rest need the per-row
+// compare. List form (list_off >= 0, items whose rows see a Gen Image hole): the item
+// processes the n_total key blocks listed at kblocks[list_off ...], each entry
+// kb | class << 24 with class an hgx_tile_class (FULL or PARTIAL; skipped blocks are not
+// listed).
+// Split items (part >= 0, prefix form only): the key blocks of one (query block, KV head)
+// are divided between two work items that may run on different CTAs; each writes its
+// unnormalised O, row maximum and row sum to partial-result slot `part`, and a combine
+// kernel merges the two slots into out.
 struct WorkItem {
   int32_t q0;        // packed index of the first query token
   int32_t kv0;       // packed index of the batch element's first token
@@ -38,8 +43,11 @@ struct WorkItem {
   int32_t n_total;   // key blocks to process
   int32_t list_off;  // -1: prefix form; else offset into the key-block list
   int32_t first;     // rows before this local row are not written (cached prefix)
+  int32_t kb0 = 0;   // prefix form: first key block processed
+  int32_t part = -1; // -1: writes out; else its partial-result slot
+  int32_t pad[2] = {0, 0};
 };
-static_assert(sizeof(WorkItem) == 32, "work item layout");
+static_assert(sizeof(WorkItem) == 48, "work item layout");
 
 constexpr uint32_t kListClassShift = 24;
 constexpr uint32_t kListBlockMask = (1u << kListClassShift) - 1;
@@ -59,6 +67,10 @@ struct Plan {
   // [cta_offsets[c], cta_offsets[c + 1]) of `items`, longest first.
   int32_t grid = 0;
   std::vector<int32_t> cta_offsets;
+  // Split items (assign_ctas with splitting): split i wrote partial slots 2i and 2i + 1;
+  // splits[i] is the whole (query block, KV head) item with part = 2i.
+  std::vector<WorkItem> splits;
+  int64_t makespan = 0;  // largest CTA load of the assignment, in key blocks + overheads
 };
 
 // Checks the packed-varlen descriptor. On failure returns INVALID_ARG with *err set.
@@ -84,9 +96,20 @@ hgx_status check_first_rows(int32_t batch, const int32_t* cu_seqlens, const hgx_
 
 // Distributes plan->items over `ctas` persistent CTAs (longest-processing-time first: each
 // item, in decreasing cost, goes to the least loaded CTA; cost = key blocks + a per-item
-// overhead), reorders the items so that every CTA's list is contiguous, and sets grid and
-// cta_offsets. grid = min(ctas, number of items).
-void assign_ctas(Plan* plan, int32_t ctas);
+// overhead), reorders the items so that every CTA's list is contiguous, and sets grid,
+// cta_offsets and makespan. grid = min(ctas, number of items).
+//
+// With allow_split, a second schedule is tried: the wrap-around rule for preemptive
+// scheduling (McNaughton) -- the CTAs are filled one after the other up to a common bound,
+// and a prefix-form item that straddles a CTA's bound is split by key blocks into two
+// items, the first finishing that CTA's list and the second opening the next one. It
+// replaces the first schedule when its makespan plus kSplitPenalty is smaller.
+constexpr int64_t kItemOverhead = 2;   // loading Q and writing O: about two key blocks
+constexpr int64_t kSplitPenalty = 3;   // the combine launch, in key blocks
+// force_split (a test hook that exercises the split path on any input): every prefix-form
+// item of two or more key blocks is split into two halves, then all items are assigned
+// longest first.
+void assign_ctas(Plan* plan, int32_t ctas, bool allow_split = false, bool force_split = false);
 
 // Tile classes of every (query block, key block) of every batch element in order (after
 // a successful build_plan with the same descriptor).

@@ -1,8 +1,9 @@
 """The attention kernel's compile-time options still build for sm_100a (no GPU needed).
 
 The default build is covered by every other test; these are the alternatives kept in the
-source (two softmax warps per row, P in four parts, polynomial exp2 for part of the
-scores). Each is compiled to an object file with nvcc, in parallel.
+source (two softmax warps per row, P in four or one parts, polynomial exp2 for part of
+the scores, double-buffered Q, a one-wait epilogue, per-element masks only, no next-item
+prefetch). Each is compiled to an object file with nvcc, in parallel.
 """
 import os
 import shutil
@@ -20,6 +21,10 @@ OPTIONS = {
     "p_in_four_parts": ["-DHGX_P_PARTS=4"],
     "p_in_one_part": ["-DHGX_P_PARTS=1"],
     "polynomial_exp2": ["-DHGX_EXP_POLY_MASK=0x0101"],
+    "double_buffered_q": ["-DHGX_Q_BUFS=2"],
+    "epilogue_one_wait": ["-DHGX_EPI_LOAD_ALL=1"],
+    "per_element_masks_only": ["-DHGX_MASK_FAST=0"],
+    "no_item_prefetch": ["-DHGX_ITEM_PREFETCH=0"],
 }
 
 

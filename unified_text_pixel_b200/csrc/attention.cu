@@ -90,6 +90,19 @@ static_assert(kPParts == 1 || kPParts == 2 || kPParts == 4, "P parts");
 // 1: the epilogue loads the whole O row from tensor memory with one wait and releases O to
 // the next item's PV before it stores (instead of four load-wait-store rounds)
 constexpr bool kEpiLoadAll = HGX_EPI_LOAD_ALL != 0;
+#ifndef HGX_MASK_FAST
+#define HGX_MASK_FAST 1
+#endif
+// 1: in a PARTIAL block, a warp whose rows are each either fully visible or fully masked
+// (e.g. a causal text row that shares its item with generation rows) skips the
+// per-element mask; its fully masked rows exponentiate with scale 0 and shift -inf
+constexpr bool kMaskFast = HGX_MASK_FAST != 0;
+#ifndef HGX_ITEM_PREFETCH
+#define HGX_ITEM_PREFETCH 1
+#endif
+// 1: the producer prefetches the next item's Q into L2 and loads the next item's first K
+// and V before it waits for the Q buffer
+constexpr bool kItemPrefetch = HGX_ITEM_PREFETCH != 0;
 constexpr uint32_t kTileBytes = 32768;        // 128 rows x 128 bf16
 constexpr uint32_t kHalfBytes = 16384;        // 128 rows x 64 bf16 (one 128-byte swizzle span)
 constexpr uint32_t kQBytes = 2 * kTileBytes;  // both Q tiles of an item
@@ -280,10 +293,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t pos = 0, q_loads = 0;
         uint32_t loaded = 0, last_par = 0;  // per slot: ever loaded, parity of its last load
         bool ok = true;
+        // K_j then V_j of block j of an item into the next two ring slots
+        auto load_kv = [&](const WorkItem& it, int j) {
+          for (int kv = 0; ok && kv < 2; ++kv) {
+            const uint32_t slot = pos % kStages;
+            const uint32_t round = pos / kStages;
+            ok = wait_bounded(c, bar_addr(c, BAR_KV_EMPTY + slot), (round & 1u) ^ 1u, SITE_PRODUCER);
+            if (!ok) break;
+            const uint32_t full = bar_addr(c, BAR_KV_FULL + slot);
+            mbar_arrive_expect_tx(full, kTileBytes);
+            const CUtensorMap* map = kv == 0 ? &tmap_k : &tmap_v;
+            const int32_t kb =
+                it.list_off < 0 ? it.kb0 + j : static_cast<int32_t>(p.kblocks[it.list_off + j] & kListBlockMask);
+            for (int hf = 0; hf < 2; ++hf)
+              tma_load_3d(sRing + slot * kTileBytes + hf * kHalfBytes, map, full, 64 * hf, it.g,
+                          it.kv0 + 128 * kb);
+            loaded |= 1u << slot;
+            last_par = (last_par & ~(1u << slot)) | ((round & 1u) << slot);
+            ++pos;
+          }
+        };
         for (int w = first_item(p); ok && w < end_item(p); w = next_item(p, w)) {
           const WorkItem it = p.items[w];
           const uint32_t qb = q_loads % kQBufs;  // Q buffer of this item
+          int j0 = 0;
           if (q_loads >= static_cast<uint32_t>(kQBufs)) {
+            // the buffer still holds an earlier item's Q: start this item's first K and V
+            // meanwhile (the ring slots free up as the previous item's last blocks retire)
+            if constexpr (kItemPrefetch) {
+              if (it.n_total > 0) load_kv(it, 0);
+              j0 = 1;
+              if (!ok) break;
+            }
             ok = wait_bounded(c, bar_addr(c, BAR_Q_EMPTY + qb), ((q_loads / kQBufs) - 1) & 1u, SITE_PRODUCER);
             if (!ok) break;
           }
@@ -297,26 +338,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                           64 * hf, 4 * it.g, t0);
           }
           ++q_loads;
-          for (int j = 0; ok && j < it.n_total; ++j) {
-            for (int kv = 0; kv < 2; ++kv) {  // K_j then V_j
-              const uint32_t slot = pos % kStages;
-              const uint32_t round = pos / kStages;
-              ok = wait_bounded(c, bar_addr(c, BAR_KV_EMPTY + slot), (round & 1u) ^ 1u,
-                                SITE_PRODUCER);
-              if (!ok) break;
-              const uint32_t full = bar_addr(c, BAR_KV_FULL + slot);
-              mbar_arrive_expect_tx(full, kTileBytes);
-              const CUtensorMap* map = kv == 0 ? &tmap_k : &tmap_v;
-              const int32_t kb =
-                it.list_off < 0 ? it.kb0 + j : static_cast<int32_t>(p.kblocks[it.list_off + j] & kListBlockMask);
-            for (int hf = 0; hf < 2; ++hf)
-                tma_load_3d(sRing + slot * kTileBytes + hf * kHalfBytes, map, full, 64 * hf, it.g,
-                            it.kv0 + 128 * kb);
-              loaded |= 1u << slot;
-              last_par = (last_par & ~(1u << slot)) | ((round & 1u) << slot);
-              ++pos;
+          if constexpr (kItemPrefetch) {  // the next item's Q into L2, one item ahead
+            const int wn = next_item(p, w);
+            if (wn < end_item(p)) {
+              const WorkItem nx = p.items[wn];
+              for (int x = 0; x < 2; ++x)
+                for (int hf = 0; hf < 2; ++hf)
+                  tma_prefetch_l2_3d(&tmap_q, 64 * hf, 4 * nx.g, min(nx.q0 + 32 * x, p.total_tokens - 1));
             }
           }
+          for (int j = j0; ok && j < it.n_total; ++j) load_kv(it, j);
         }
         // drain: every load this thread issued must land before the CTA exits (on the normal
         // path they all have, and these waits return at once)
@@ -514,10 +545,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int ch = 0; ch < kCols / 32; ++ch)
 #pragma unroll
           for (int e = 0; e < 32; ++e) s[32 * ch + e] = __uint_as_float(sr[ch][e]);
+        bool dead = false;  // every key of this block is masked for this row (kMaskFast)
         if (!full) {
           // keys [0, nvis) of this block are in the prefix
           const int nvis = row_lim - 128 * kb - kCols * half;
-          if (hbase >= 0) {
+          // a block that runs past the element's end holds another element's keys (or the
+          // zero fill past T): those are always masked one by one
+          const bool past_end = 128 * kb + 128 > it.len;
+          const bool need_mask = hbase >= 0 || (nvis < kCols && (nvis > 0 || past_end));
+          if (kMaskFast && !__any_sync(0xffffffffu, need_mask)) {
+            dead = nvis <= 0;
+          } else if (hbase >= 0) {
             // keys hidden by Gen Image holes: the mask words of this thread's columns, picked
             // up front so that every index below is a compile-time constant
             uint32_t hw[kCols / 32];
@@ -550,6 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float mx = m8[0];
 #pragma unroll
         for (int i = 1; i < kCols / 16; ++i) mx = fmaxf(mx, m8[i]);
+        if (dead) mx = -INFINITY;
         if constexpr (kSplit == 2) {
           // exchange with the other half of the row; the barrier also decides, for the
           // whole tile, whether every wait succeeded
@@ -579,7 +618,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // a row whose keys so far were all hidden (a Gen Image hole before its first visible
         // key) still has m_used = -inf: exponentiate against 0, so its masked scores give
         // exact zeros and its first real maximum later rescales the all-zero O by 0
-        const float mb = m_used == -INFINITY ? 0.f : m_used * sl2;
+        // a row that sees no key of this block: scale 0 and shift -inf give exact zeros (its
+        // scores are finite: the block lies inside its element)
+        const float mb = dead ? INFINITY : m_used == -INFINITY ? 0.f : m_used * sl2;
+        const float sl2_row = dead ? 0.f : sl2;
         // exponentials and P. With one warp per row, P is written in kPParts parts and each
         // part but the last is published before the next is exponentiated, so that the PV
         // MMAs of the early parts overlap the later exponentials -- unless O must be rescaled
@@ -596,9 +638,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto exp_part = [&](auto from_c, auto to_c) {
           constexpr int kFrom = decltype(from_c)::value, kTo = decltype(to_c)::value;
           if (kExpPolyOn && full)
-            exp_store_p<true, kCols, kFrom, kTo>(s, sl2, mb, tP, acc);  // no -inf: polynomial allowed
+            exp_store_p<true, kCols, kFrom, kTo>(s, sl2_row, mb, tP, acc);  // no -inf: polynomial allowed
           else
-            exp_store_p<false, kCols, kFrom, kTo>(s, sl2, mb, tP, acc);  // MUFU: zeros for -inf
+            exp_store_p<false, kCols, kFrom, kTo>(s, sl2_row, mb, tP, acc);  // MUFU: zeros for -inf
         };
         exp_part(std::integral_constant<int, 0>{}, std::integral_constant<int, kW>{});
         if constexpr (kParts >= 2) {

@@ -246,11 +246,12 @@ hgx_status hgx_attn_visible_pairs(int32_t batch, const int32_t* cu_seqlens_host,
  * work item in execution order, (cta, q0, kv_head, kb0, n_total, part, n_full, list_off).
  * A work item covers 64 query tokens x the 4 query heads of one KV head; it processes key
  * blocks kb0 .. kb0 + n_total - 1 (prefix form, list_off < 0) or the n_total blocks of its
- * key-block list (list form). part >= 0 marks one of the two halves of a split item, which
- * write partial results that a combine kernel merges. mode 0: the library's own policy;
- * 1: the wrap-around schedule with split items is taken whenever its makespan plus the
- * combine's cost is smaller; 2: as under HGX_DEBUG_SPLIT_TEST (every prefix-form item of
- * two or more key blocks split in two). out has room for cap items (8 int32 each);
+ * key-block list (list form). part >= 0 marks one of the parts of a split item (slots of
+ * one item are consecutive), which write partial results that a combine kernel merges.
+ * mode 0: the library's own policy; 1: the CTAs loaded above the mean hand their last items
+ * out in parts to the least-loaded CTAs whenever that lowers the makespan by more than the
+ * combine's cost; 2: as under HGX_DEBUG_SPLIT_TEST (every prefix-form item of two or more
+ * key blocks split in two). out has room for cap items (8 int32 each);
  * *n_items receives the count; out may be NULL to query the count. */
 hgx_status hgx_attn_schedule(int32_t batch, const int32_t* cu_seqlens_host,
                              const hgx_segment* segs_host, const int32_t* cu_segs_host,

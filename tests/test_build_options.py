@@ -2,8 +2,7 @@
 
 The default build is covered by every other test; these are the alternatives kept in the
 source (two softmax warps per row, P in four or one parts, polynomial exp2 for part of
-the scores, double-buffered Q, a one-wait epilogue, per-element masks only, no next-item
-prefetch). Each is compiled to an object file with nvcc, in parallel.
+the scores, direct epilogue stores, no split items). Each is compiled to an object file with nvcc, in parallel.
 """
 import os
 import shutil
@@ -21,10 +20,8 @@ OPTIONS = {
     "p_in_four_parts": ["-DHGX_P_PARTS=4"],
     "p_in_one_part": ["-DHGX_P_PARTS=1"],
     "polynomial_exp2": ["-DHGX_EXP_POLY_MASK=0x0101"],
-    "double_buffered_q": ["-DHGX_Q_BUFS=2"],
-    "epilogue_one_wait": ["-DHGX_EPI_LOAD_ALL=1"],
-    "per_element_masks_only": ["-DHGX_MASK_FAST=0"],
-    "no_item_prefetch": ["-DHGX_ITEM_PREFETCH=0"],
+    "no_split_items": ["-DHGX_SPLIT_KV=0"],
+    "direct_epilogue_stores": ["-DHGX_EPI_TMA=0"],
 }
 
 
@@ -35,8 +32,9 @@ def test_attention_options_compile():
     with tempfile.TemporaryDirectory() as tmp:
         procs = {}
         for name, flags in OPTIONS.items():
+            target = os.path.join(CSRC, "api.cu") if "SPLIT_KV" in flags[0] else src
             cmd = [nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17",
-                   "-I", CSRC, *flags, "-c", src, "-o", os.path.join(tmp, name + ".o")]
+                   "-I", CSRC, *flags, "-c", target, "-o", os.path.join(tmp, name + ".o")]
             procs[name] = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT)
         failed = {}
         for name, proc in procs.items():

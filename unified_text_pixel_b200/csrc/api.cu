@@ -70,7 +70,7 @@ struct hgx_attn_handle {
 namespace {
 
 #ifndef HGX_SPLIT_KV
-#define HGX_SPLIT_KV 0
+#define HGX_SPLIT_KV 1
 #endif
 // 1: the planner may split items by key blocks when that balances the persistent CTAs
 // better (hgx::assign_ctas); 0: longest-processing-time assignment only
@@ -241,7 +241,8 @@ hgx_status prepare_plan(hgx_attn_handle* h, cudaStream_t stream, int32_t batch,
     need += (u.bytes + 255) & ~size_t(255);
   }
   // partial results of split items (written and read on the device only)
-  const size_t slots = 2 * pl.splits.size();
+  size_t slots = 0;
+  for (const hgx::WorkItem& sp : pl.splits) slots += static_cast<size_t>(sp.n_parts);
   const size_t partial_bytes =
       slots * (hgx::kPartialSlotFloats * sizeof(float) + hgx::kPartialSlotRows * sizeof(float2));
   if (partial_bytes > h->partial_cap) {
@@ -303,9 +304,9 @@ hgx_status finish(hgx_attn_handle* h, cudaStream_t stream) {
 hgx_status run_attention(hgx_attn_handle* h, cudaStream_t stream, const void* q, const void* k,
                          const void* v, void* out) {
   const int32_t T = h->plan.total_tokens;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   if (!make_map(&mq, q, 32, T, 4, hgx::kTileTokens) || !make_map(&mk, k, 8, T, 1, 128) ||
-      !make_map(&mv, v, 8, T, 1, 128))
+      !make_map(&mv, v, 8, T, 1, 128) || !make_map(&mo, out, 32, T, 4, 8))
     return fail(h, HGX_ERR_CUDA, "cuTensorMapEncodeTiled failed");
   hgx::AttnParams p{};
   p.items = h->d_items;
@@ -317,7 +318,9 @@ hgx_status run_attention(hgx_attn_handle* h, cudaStream_t stream, const void* q,
   p.hole_base = h->plan.has_holes ? h->d_hole_base : nullptr;
   p.hole_masks = h->plan.has_holes ? h->d_hole_masks : nullptr;
   p.out = out;
-  const size_t slots = 2 * h->plan.splits.size();
+  p.out_tma = 1;
+  size_t slots = 0;
+  for (const hgx::WorkItem& sp : h->plan.splits) slots += static_cast<size_t>(sp.n_parts);
   p.partial_o = slots ? static_cast<float*>(h->d_partial) : nullptr;
   p.partial_ml = slots ? reinterpret_cast<float2*>(static_cast<float*>(h->d_partial) +
                                                    slots * hgx::kPartialSlotFloats)
@@ -326,7 +329,7 @@ hgx_status run_attention(hgx_attn_handle* h, cudaStream_t stream, const void* q,
   p.flags = h->flags;
   p.err = h->d_err;
   p.wait_limit_ns = h->wait_limit_ns;
-  cudaError_t e = hgx::launch_attention(stream, mq, mk, mv, p, h->plan.grid);
+  cudaError_t e = hgx::launch_attention(stream, mq, mk, mv, mo, p, h->plan.grid);
   if (e != cudaSuccess) return cuda_fail(h, e, "attention launch");
   if (slots) {
     e = hgx::launch_combine(stream, h->d_splits, static_cast<int32_t>(h->plan.splits.size()), p.partial_o,

@@ -66,15 +66,11 @@ constexpr int kThreads = 128 + 2 * kSoftmaxThreads;
 // register budgets after setmaxnreg (launch: 384 x 168 or 640 x 96 registers)
 constexpr uint32_t kRegsLow = kSplit == 1 ? 120 : 64;   // producer/MMA warpgroup
 constexpr uint32_t kRegsHigh = kSplit == 1 ? 192 : 104;  // softmax warpgroups
-#ifndef HGX_Q_BUFS
-#define HGX_Q_BUFS 1
-#endif
-// Q buffers (each both Q tiles of an item): 2 loads the next item's Q during the current
-// item, which leaves room for 3 K/V slots only
-constexpr int kQBufs = HGX_Q_BUFS;
-static_assert(kQBufs == 1 || kQBufs == 2, "Q buffers");
+// One Q buffer (both Q tiles of an item): a second one, to load the next item's Q during
+// the current item, leaves room for 3 K/V slots only and measured slower.
+constexpr int kQBufs = 1;
 #ifndef HGX_KV_STAGES
-#define HGX_KV_STAGES (HGX_Q_BUFS == 2 ? 3 : 4)
+#define HGX_KV_STAGES 4
 #endif
 constexpr int kStages = HGX_KV_STAGES;        // K/V ring slots
 #ifndef HGX_P_PARTS
@@ -84,25 +80,6 @@ constexpr int kStages = HGX_KV_STAGES;        // K/V ring slots
 // that the PV MMAs of the first parts overlap the exponentials of the later ones
 constexpr int kPParts = HGX_P_PARTS;
 static_assert(kPParts == 1 || kPParts == 2 || kPParts == 4, "P parts");
-#ifndef HGX_EPI_LOAD_ALL
-#define HGX_EPI_LOAD_ALL 0
-#endif
-// 1: the epilogue loads the whole O row from tensor memory with one wait and releases O to
-// the next item's PV before it stores (instead of four load-wait-store rounds)
-constexpr bool kEpiLoadAll = HGX_EPI_LOAD_ALL != 0;
-#ifndef HGX_MASK_FAST
-#define HGX_MASK_FAST 1
-#endif
-// 1: in a PARTIAL block, a warp whose rows are each either fully visible or fully masked
-// (e.g. a causal text row that shares its item with generation rows) skips the
-// per-element mask; its fully masked rows exponentiate with scale 0 and shift -inf
-constexpr bool kMaskFast = HGX_MASK_FAST != 0;
-#ifndef HGX_ITEM_PREFETCH
-#define HGX_ITEM_PREFETCH 1
-#endif
-// 1: the producer prefetches the next item's Q into L2 and loads the next item's first K
-// and V before it waits for the Q buffer
-constexpr bool kItemPrefetch = HGX_ITEM_PREFETCH != 0;
 constexpr uint32_t kTileBytes = 32768;        // 128 rows x 128 bf16
 constexpr uint32_t kHalfBytes = 16384;        // 128 rows x 64 bf16 (one 128-byte swizzle span)
 constexpr uint32_t kQBytes = 2 * kTileBytes;  // both Q tiles of an item
@@ -128,7 +105,17 @@ constexpr uint32_t kMiscOffset = kBarOffset + 8 * BAR_COUNT;  // tmem base, abor
 // [iteration parity][tile][half][row] floats
 constexpr uint32_t kXchgOffset = kMiscOffset + 16;
 constexpr uint32_t kXchgBytes = kSplit == 2 ? 2 * 2 * 2 * 128 * 4 : 0;
-constexpr uint32_t kSmemUsed = kXchgOffset + kXchgBytes;
+#ifndef HGX_EPI_TMA
+#define HGX_EPI_TMA 1
+#endif
+// 1: the epilogue writes O through shared memory with TMA tensor stores: each softmax warp
+// stages its 8 tokens x 4 heads x 64 features (4 KB, 128-byte swizzle) and one lane stores
+// the box, so that global memory sees whole lines (a warp's direct 16-byte stores touch 32
+// rows 256 B apart). Warps with a row outside the element's written range store directly.
+constexpr bool kEpiTma = HGX_EPI_TMA != 0 && kSplit == 1;
+constexpr uint32_t kEpiOffset = (kXchgOffset + kXchgBytes + 1023u) & ~1023u;
+constexpr uint32_t kEpiBytes = kEpiTma ? 8 * 4096 : 0;  // one 4 KB box per softmax warp
+constexpr uint32_t kSmemUsed = kEpiOffset + kEpiBytes;
 constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // slack to align the base to 1024 B
 static_assert(kSmemBytes <= 232448, "more dynamic shared memory than an sm_100 CTA may have");
 
@@ -226,7 +213,8 @@ __device__ __forceinline__ int next_item(const AttnParams& p, int w) {
 __global__ void __launch_bounds__(kThreads, 1)
     attention_kernel(const __grid_constant__ CUtensorMap tmap_q,
                      const __grid_constant__ CUtensorMap tmap_k,
-                     const __grid_constant__ CUtensorMap tmap_v, const AttnParams p) {
+                     const __grid_constant__ CUtensorMap tmap_v,
+                     const __grid_constant__ CUtensorMap tmap_out, const AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;  // 128-byte swizzle wants 1024-B alignment
@@ -316,15 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int w = first_item(p); ok && w < end_item(p); w = next_item(p, w)) {
           const WorkItem it = p.items[w];
           const uint32_t qb = q_loads % kQBufs;  // Q buffer of this item
-          int j0 = 0;
           if (q_loads >= static_cast<uint32_t>(kQBufs)) {
-            // the buffer still holds an earlier item's Q: start this item's first K and V
-            // meanwhile (the ring slots free up as the previous item's last blocks retire)
-            if constexpr (kItemPrefetch) {
-              if (it.n_total > 0) load_kv(it, 0);
-              j0 = 1;
-              if (!ok) break;
-            }
             ok = wait_bounded(c, bar_addr(c, BAR_Q_EMPTY + qb), ((q_loads / kQBufs) - 1) & 1u, SITE_PRODUCER);
             if (!ok) break;
           }
@@ -338,16 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                           64 * hf, 4 * it.g, t0);
           }
           ++q_loads;
-          if constexpr (kItemPrefetch) {  // the next item's Q into L2, one item ahead
-            const int wn = next_item(p, w);
-            if (wn < end_item(p)) {
-              const WorkItem nx = p.items[wn];
-              for (int x = 0; x < 2; ++x)
-                for (int hf = 0; hf < 2; ++hf)
-                  tma_prefetch_l2_3d(&tmap_q, 64 * hf, 4 * nx.g, min(nx.q0 + 32 * x, p.total_tokens - 1));
-            }
-          }
-          for (int j = j0; ok && j < it.n_total; ++j) load_kv(it, j);
+          for (int j = 0; ok && j < it.n_total; ++j) load_kv(it, j);
         }
         // drain: every load this thread issued must land before the CTA exits (on the normal
         // path they all have, and these waits return at once)
@@ -545,17 +516,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int ch = 0; ch < kCols / 32; ++ch)
 #pragma unroll
           for (int e = 0; e < 32; ++e) s[32 * ch + e] = __uint_as_float(sr[ch][e]);
-        bool dead = false;  // every key of this block is masked for this row (kMaskFast)
         if (!full) {
           // keys [0, nvis) of this block are in the prefix
           const int nvis = row_lim - 128 * kb - kCols * half;
-          // a block that runs past the element's end holds another element's keys (or the
-          // zero fill past T): those are always masked one by one
-          const bool past_end = 128 * kb + 128 > it.len;
-          const bool need_mask = hbase >= 0 || (nvis < kCols && (nvis > 0 || past_end));
-          if (kMaskFast && !__any_sync(0xffffffffu, need_mask)) {
-            dead = nvis <= 0;
-          } else if (hbase >= 0) {
+          if (hbase >= 0) {
             // keys hidden by Gen Image holes: the mask words of this thread's columns, picked
             // up front so that every index below is a compile-time constant
             uint32_t hw[kCols / 32];
@@ -588,7 +552,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         float mx = m8[0];
 #pragma unroll
         for (int i = 1; i < kCols / 16; ++i) mx = fmaxf(mx, m8[i]);
-        if (dead) mx = -INFINITY;
         if constexpr (kSplit == 2) {
           // exchange with the other half of the row; the barrier also decides, for the
           // whole tile, whether every wait succeeded
@@ -618,10 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // a row whose keys so far were all hidden (a Gen Image hole before its first visible
         // key) still has m_used = -inf: exponentiate against 0, so its masked scores give
         // exact zeros and its first real maximum later rescales the all-zero O by 0
-        // a row that sees no key of this block: scale 0 and shift -inf give exact zeros (its
-        // scores are finite: the block lies inside its element)
-        const float mb = dead ? INFINITY : m_used == -INFINITY ? 0.f : m_used * sl2;
-        const float sl2_row = dead ? 0.f : sl2;
+        const float mb = m_used == -INFINITY ? 0.f : m_used * sl2;
         // exponentials and P. With one warp per row, P is written in kPParts parts and each
         // part but the last is published before the next is exponentiated, so that the PV
         // MMAs of the early parts overlap the later exponentials -- unless O must be rescaled
@@ -638,9 +598,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto exp_part = [&](auto from_c, auto to_c) {
           constexpr int kFrom = decltype(from_c)::value, kTo = decltype(to_c)::value;
           if (kExpPolyOn && full)
-            exp_store_p<true, kCols, kFrom, kTo>(s, sl2_row, mb, tP, acc);  // no -inf: polynomial allowed
+            exp_store_p<true, kCols, kFrom, kTo>(s, sl2, mb, tP, acc);  // no -inf: polynomial allowed
           else
-            exp_store_p<false, kCols, kFrom, kTo>(s, sl2_row, mb, tP, acc);  // MUFU: zeros for -inf
+            exp_store_p<false, kCols, kFrom, kTo>(s, sl2, mb, tP, acc);  // MUFU: zeros for -inf
         };
         exp_part(std::integral_constant<int, 0>{}, std::integral_constant<int, kW>{});
         if constexpr (kParts >= 2) {
@@ -723,31 +683,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
       const float inv_l = 1.0f / l;
-      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) +
-                           (static_cast<size_t>(tok) * 32 + head) * 128 + kCols * half;
-      if constexpr (kEpiLoadAll) {
-        // every tensor-memory load of the row first, one wait, then the stores
-        uint32_t o[kCols / 32][32];
+      if (kEpiTma && p.out_tma && __all_sync(0xffffffffu, valid)) {
+        // stage this warp's 32 rows = 8 tokens x 4 heads, 64 features at a time, in the
+        // 128-byte-swizzled box layout (row = lane, 16-byte chunk j at j ^ (lane & 7)), and
+        // store each box with one TMA store
+        const uint32_t stage = base + kEpiOffset + ((warp - 4) & 7) * 4096u;
+        uint8_t* stage_g = gbase + kEpiOffset + ((warp - 4) & 7) * 4096u;
+        const int32_t tok0 = it.q0 + 32 * x + 8 * quarter;
 #pragma unroll
-        for (int ch = 0; ch < kCols / 32; ++ch) tmem_ld32(tO + 32 * ch, o[ch]);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(bar_addr(c, BAR_O_EMPTY + x));  // O is in registers: the next PV may start
-        if (valid) {
+        for (int c64 = 0; c64 < 2; ++c64) {
+          uint32_t o[2][32];
+          tmem_ld32(tO + 64 * c64, o[0]);
+          tmem_ld32(tO + 64 * c64 + 32, o[1]);
+          tmem_wait_ld();
+          // the warp's previous box (the first half, or the last item's second half) must
+          // have left shared memory before it is overwritten
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
 #pragma unroll
-          for (int ch = 0; ch < kCols / 32; ++ch) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * ch);
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              d4[e] = make_uint4(
-                  pack_bf16x2(__uint_as_float(o[ch][8 * e]) * inv_l, __uint_as_float(o[ch][8 * e + 1]) * inv_l),
-                  pack_bf16x2(__uint_as_float(o[ch][8 * e + 2]) * inv_l, __uint_as_float(o[ch][8 * e + 3]) * inv_l),
-                  pack_bf16x2(__uint_as_float(o[ch][8 * e + 4]) * inv_l, __uint_as_float(o[ch][8 * e + 5]) * inv_l),
-                  pack_bf16x2(__uint_as_float(o[ch][8 * e + 6]) * inv_l, __uint_as_float(o[ch][8 * e + 7]) * inv_l));
+          for (int j = 0; j < 8; ++j) {
+            const uint32_t* w = o[j >> 2] + 8 * (j & 3);
+            const uint4 v = make_uint4(pack_bf16x2(__uint_as_float(w[0]) * inv_l, __uint_as_float(w[1]) * inv_l),
+                                       pack_bf16x2(__uint_as_float(w[2]) * inv_l, __uint_as_float(w[3]) * inv_l),
+                                       pack_bf16x2(__uint_as_float(w[4]) * inv_l, __uint_as_float(w[5]) * inv_l),
+                                       pack_bf16x2(__uint_as_float(w[6]) * inv_l, __uint_as_float(w[7]) * inv_l));
+            *reinterpret_cast<uint4*>(stage_g + lane * 128 + ((j ^ (lane & 7)) << 4)) = v;
+          }
+          fence_proxy_async_smem();  // the TMA reads the staged box through the async proxy
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&tmap_out, stage, 64 * c64, 4 * it.g, tok0);
+            bulk_commit_group();
           }
         }
+        tc_fence_before();
+        mbar_arrive(bar_addr(c, BAR_O_EMPTY + x));
         continue;
       }
+      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.out) +
+                           (static_cast<size_t>(tok) * 32 + head) * 128 + kCols * half;
 #pragma unroll
       for (int ch = 0; ch < kCols / 32; ++ch) {
         uint32_t o[32];
@@ -768,12 +742,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar_addr(c, BAR_O_EMPTY + x));
     }
+    if (kEpiTma && lane == 0) bulk_wait_all();  // this warp's box stores have completed
     tc_fence_before();
     named_bar_sync(1, kThreads);  // pairs with the producer/MMA warpgroup's barrier
   }
 }
 
-// One warp per row of a split item: lane i merges features 4i .. 4i + 3.
+// One warp per row of a split item: lane i merges features 4i .. 4i + 3 over the item's
+// n_parts partial results, out = sum_p O_p 2^(M_p - M) / sum_p l_p 2^(M_p - M), M = max M_p.
 __global__ void __launch_bounds__(256) combine_kernel(const WorkItem* __restrict__ splits, int32_t n_splits,
                                                       const float* __restrict__ po,
                                                       const float2* __restrict__ pml, __nv_bfloat16* out) {
@@ -784,17 +760,28 @@ __global__ void __launch_bounds__(256) combine_kernel(const WorkItem* __restrict
   const int x = (gw >> 7) & 1, row = gw & 127;
   const int32_t tok = it.q0 + 32 * x + (row >> 2);
   if (!(tok - it.kv0 < it.len && tok - it.kv0 >= it.first)) return;
-  const size_t ra = (static_cast<size_t>(it.part) * 2 + x) * 128 + row;
-  const size_t rb = ra + kPartialSlotRows;  // slot part + 1
-  const float2 a = pml[ra], b = pml[rb];
-  const float m = fmaxf(a.x, b.x);  // finite: every written row sees at least itself
-  const float wa = a.y > 0.f ? exp2f(a.x - m) : 0.f;
-  const float wb = b.y > 0.f ? exp2f(b.x - m) : 0.f;
-  const float inv = 1.f / (a.y * wa + b.y * wb);
-  const float4 oa = reinterpret_cast<const float4*>(po + ra * 128)[lane];
-  const float4 ob = reinterpret_cast<const float4*>(po + rb * 128)[lane];
-  const uint32_t lo = pack_bf16x2((oa.x * wa + ob.x * wb) * inv, (oa.y * wa + ob.y * wb) * inv);
-  const uint32_t hi = pack_bf16x2((oa.z * wa + ob.z * wb) * inv, (oa.w * wa + ob.w * wb) * inv);
+  auto prow = [&](int i) { return (static_cast<size_t>(it.part + i) * 2 + x) * 128 + row; };
+  float m = -INFINITY;
+  for (int i = 0; i < it.n_parts; ++i) {
+    const float2 ml = pml[prow(i)];
+    if (ml.y > 0.f) m = fmaxf(m, ml.x);  // finite: every written row sees at least itself
+  }
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float den = 0.f;
+  for (int i = 0; i < it.n_parts; ++i) {
+    const float2 ml = pml[prow(i)];
+    if (!(ml.y > 0.f)) continue;  // the row saw no key of this part
+    const float wgt = exp2f(ml.x - m);
+    const float4 o = reinterpret_cast<const float4*>(po + prow(i) * 128)[lane];
+    acc.x = fmaf(o.x, wgt, acc.x);
+    acc.y = fmaf(o.y, wgt, acc.y);
+    acc.z = fmaf(o.z, wgt, acc.z);
+    acc.w = fmaf(o.w, wgt, acc.w);
+    den = fmaf(ml.y, wgt, den);
+  }
+  const float inv = 1.f / den;
+  const uint32_t lo = pack_bf16x2(acc.x * inv, acc.y * inv);
+  const uint32_t hi = pack_bf16x2(acc.z * inv, acc.w * inv);
   const int32_t head = 4 * it.g + (row & 3);
   reinterpret_cast<uint2*>(out + (static_cast<size_t>(tok) * 32 + head) * 128)[lane] = make_uint2(lo, hi);
 }
@@ -814,7 +801,7 @@ size_t attention_smem_bytes() { return kSmemBytes; }
 
 cudaError_t launch_attention(cudaStream_t stream, const CUtensorMap& tmap_q,
                              const CUtensorMap& tmap_k, const CUtensorMap& tmap_v,
-                             const AttnParams& p, int grid) {
+                             const CUtensorMap& tmap_out, const AttnParams& p, int grid) {
   static uint64_t configured = 0;  // bit per device: shared-memory limit raised
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -825,7 +812,7 @@ cudaError_t launch_attention(cudaStream_t stream, const CUtensorMap& tmap_q,
     if (e != cudaSuccess) return e;
     if (dev < 64) configured |= 1ull << dev;
   }
-  attention_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tmap_q, tmap_k, tmap_v, p);
+  attention_kernel<<<grid, kThreads, kSmemBytes, stream>>>(tmap_q, tmap_k, tmap_v, tmap_out, p);
   return cudaGetLastError();
 }
 

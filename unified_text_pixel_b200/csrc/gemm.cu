@@ -31,6 +31,10 @@ namespace {
 using namespace sm100;
 using namespace waits;
 
+#ifndef HGX_GEMM_L2_HINTS
+#define HGX_GEMM_L2_HINTS 1
+#endif
+constexpr bool kL2Hints = HGX_GEMM_L2_HINTS != 0;  // L2 cache policies on the operand loads
 constexpr int kThreads = 192;
 constexpr int BM = 128, BN = 256, BK = 64, kStages = 4;
 constexpr uint32_t kABytes = BM * BK * 2;  // 16 KB
@@ -136,6 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tmap_a);
       tma_prefetch_desc(&tmap_b);
+      const uint64_t pol_a = l2_policy_evict_first(), pol_b = l2_policy_evict_last();
       uint32_t pos = 0, loaded = 0, last_par = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < n_tiles_total; t += gridDim.x) {
@@ -146,8 +151,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t full = bar_addr(c, G_FULL + slot);
           mbar_arrive_expect_tx(full, kStageBytes);
           const uint32_t sa = base + slot * kStageBytes;
-          tma_load_2d(sa, &tmap_a, full, kb * BK, m0);
-          tma_load_2d(sa + kABytes, &tmap_b, full, kb * BK, n0);
+          if constexpr (kL2Hints) {
+            // the weights (B) are read again by every row block: keep them in L2; the
+            // activations (A) are read by the column tiles of their row block at about the
+            // same time and then never again
+            tma_load_2d_hint(sa, &tmap_a, full, kb * BK, m0, pol_a);
+            tma_load_2d_hint(sa + kABytes, &tmap_b, full, kb * BK, n0, pol_b);
+          } else {
+            tma_load_2d(sa, &tmap_a, full, kb * BK, m0);
+            tma_load_2d(sa + kABytes, &tmap_b, full, kb * BK, n0);
+          }
           loaded |= 1u << slot;
           last_par = (last_par & ~(1u << slot)) | ((round & 1u) << slot);
           ++pos;

@@ -33,6 +33,7 @@ struct AttnParams {
   const int32_t* hole_base;    // [T] row's first hole-mask index, -1 = none (holes only)
   const uint32_t* hole_masks;  // 4 words per (segment, key block): hidden keys (holes only)
   void* out;               // bf16 [T, 32, 128]
+  uint32_t out_tma;        // 1: tmap_out describes out (epilogue TMA stores)
   float* partial_o;        // split items: unnormalised O per slot, fp32 [slots][2][128][128]
   float2* partial_ml;      // split items: (row maximum x scale log2 e, row sum) [slots][2][128]
   float scale_log2;        // softmax scale * log2(e)
@@ -41,8 +42,9 @@ struct AttnParams {
   uint64_t wait_limit_ns;  // bound of every wait
 };
 
-// Merges the two partial results of every split item into out (bf16):
-// out = (O_a 2^(M_a - M) + O_b 2^(M_b - M)) / (l_a 2^(M_a - M) + l_b 2^(M_b - M)), M = max.
+// Merges the partial results of every split item into out (bf16):
+// out = sum_p O_p 2^(M_p - M) / sum_p l_p 2^(M_p - M), M = the largest M_p of the parts the
+// row saw keys in.
 cudaError_t launch_combine(cudaStream_t stream, const WorkItem* splits, int32_t n_splits,
                            const float* partial_o, const float2* partial_ml, void* out);
 constexpr size_t kPartialSlotFloats = 2 * 128 * 128;  // fp32 O of one slot
@@ -51,9 +53,11 @@ constexpr size_t kPartialSlotRows = 2 * 128;          // rows (and (M, l) pairs)
 // Bytes of dynamic shared memory the attention kernel needs.
 size_t attention_smem_bytes();
 
+// tmap_out: bf16 out [T, 32, 128] with a (64 features, 4 heads, 8 tokens) box and 128-byte
+// swizzle, used when p.out_tma is set (the epilogue's TMA stores)
 cudaError_t launch_attention(cudaStream_t stream, const CUtensorMap& tmap_q,
                              const CUtensorMap& tmap_k, const CUtensorMap& tmap_v,
-                             const AttnParams& p, int grid);
+                             const CUtensorMap& tmap_out, const AttnParams& p, int grid);
 
 struct GemmParams {
   int32_t M, N, K;           // C[M, N] = A[M, K] * B[N, K]^T; N % 256 == 0, K % 64 == 0

@@ -332,9 +332,9 @@ extern "C" hgx_status hgx_attn_forward_noalloc(const hgx_attn_config* cfg, void*
   if (hgx::launch_prologue(s, q, k, pos_thw, q_norm_w, k_norm_w, T, cfg->rms_eps, rope) != cudaSuccess)
     return HGX_ERR_CUDA;
 
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   if (!encode(&mq, q, 32, T, 4, hgx::kTileTokens) || !encode(&mk, k, 8, T, 1, 128) ||
-      !encode(&mv, v, 8, T, 1, 128))
+      !encode(&mv, v, 8, T, 1, 128) || !encode(&mo, out, 32, T, 4, 8))
     return HGX_ERR_CUDA;
   const float scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale
                                                : static_cast<float>(1.0 / std::sqrt(128.0));
@@ -345,11 +345,12 @@ extern "C" hgx_status hgx_attn_forward_noalloc(const hgx_attn_config* cfg, void*
   p.total_tokens = T;
   p.lim = d_lim;
   p.out = out;
+  p.out_tma = 1;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.flags = 0;
   p.err = d_err;
   p.wait_limit_ns = 2000000000ull;
-  if (hgx::launch_attention(s, mq, mk, mv, p, grid) != cudaSuccess) return HGX_ERR_CUDA;
+  if (hgx::launch_attention(s, mq, mk, mv, mo, p, grid) != cudaSuccess) return HGX_ERR_CUDA;
   if (!synchronize) return HGX_OK;
   if (cudaStreamSynchronize(s) != cudaSuccess) return HGX_ERR_CUDA;
   uint32_t word = 0;

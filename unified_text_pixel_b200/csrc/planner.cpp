@@ -286,55 +286,77 @@ int64_t lpt(const std::vector<WorkItem>& items, int32_t g, std::vector<int32_t>*
   return makespan;
 }
 
-// Wrap-around fill (McNaughton) up to the bound B = ceil((total cost + the overhead of up
-// to g - 1 splits) / g). Produces the items in CTA order, the offsets, the splits and the
-// makespan.
-int64_t wrap_around(const std::vector<WorkItem>& items, int32_t g, std::vector<WorkItem>* out,
-                    std::vector<int32_t>* offsets, std::vector<WorkItem>* splits) {
+// Tail split: start from the longest-first assignment; every CTA loaded above the target
+// (the mean load plus one item overhead) gives back its last -- smallest -- items as long as
+// they can be split (prefix form, two or more key blocks), and the key blocks of those items
+// are handed out in parts, each part to the least-loaded CTA as much as fits under the
+// target (at least kMinPartBlocks). An item that ends up in one part stays whole.
+constexpr int64_t kPartOverhead = 3;  // an extra item's Q load, pipeline fill and epilogue
+constexpr int32_t kMinPartBlocks = 2;
+int64_t tail_split(const std::vector<WorkItem>& items, int32_t g, const std::vector<int32_t>& owner,
+                   std::vector<std::vector<WorkItem>>* lists, std::vector<WorkItem>* splits) {
+  lists->assign(static_cast<size_t>(g), {});
+  std::vector<int64_t> load(static_cast<size_t>(g), 0);
   int64_t total = 0;
-  for (const WorkItem& it : items) total += item_cost(it);
-  const int64_t bound = (total + kItemOverhead * (g - 1) + g - 1) / g;
-  out->clear();
-  splits->clear();
-  offsets->assign(static_cast<size_t>(g) + 1, 0);
-  int32_t c = 0;
-  int64_t load = 0, makespan = 0;
-  auto close_cta = [&]() {
-    makespan = std::max(makespan, load);
-    (*offsets)[static_cast<size_t>(c) + 1] = static_cast<int32_t>(out->size());
-    ++c;
-    load = 0;
-  };
-  for (const WorkItem& it : items) {
-    const int64_t cost = item_cost(it);
-    if (c < g - 1 && load + cost > bound) {
-      const int64_t room = bound - load - kItemOverhead;  // key blocks that still fit
-      if (it.list_off < 0 && it.part < 0 && room >= 1 && it.n_total - room >= 1) {
-        const int32_t a = static_cast<int32_t>(room);
-        const int32_t slot = 2 * static_cast<int32_t>(splits->size());
-        WorkItem whole = it;
-        whole.part = slot;
-        splits->push_back(whole);
-        WorkItem head = it;  // the first key blocks: end of this CTA's list
-        head.n_total = a;
-        head.part = slot;
-        out->push_back(head);
-        load += a + kItemOverhead;
-        close_cta();
-        WorkItem tail = it;  // the rest: start of the next CTA's list
-        tail.kb0 = it.kb0 + a;
-        tail.n_total = it.n_total - a;
-        tail.part = slot + 1;
-        out->push_back(tail);
-        load = item_cost(tail);
-        continue;
-      }
-      if (load > 0) close_cta();
-    }
-    out->push_back(it);
-    load += cost;
+  for (size_t i = 0; i < items.size(); ++i) {
+    (*lists)[static_cast<size_t>(owner[i])].push_back(items[i]);
+    load[static_cast<size_t>(owner[i])] += item_cost(items[i]);
+    total += item_cost(items[i]);
   }
-  while (c < g) close_cta();
+  const int64_t target = (total + g - 1) / g + kPartOverhead;
+  std::vector<WorkItem> given;
+  for (int32_t c = 0; c < g; ++c) {
+    auto& l = (*lists)[static_cast<size_t>(c)];
+    while (load[static_cast<size_t>(c)] > target && l.size() > 1) {
+      const WorkItem& it = l.back();
+      if (it.list_off >= 0 || it.part >= 0 || it.n_total < 2 * kMinPartBlocks) break;
+      load[static_cast<size_t>(c)] -= item_cost(it);
+      given.push_back(it);
+      l.pop_back();
+    }
+  }
+  splits->clear();
+  using Load = std::pair<int64_t, int32_t>;
+  std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+  for (int32_t c = 0; c < g; ++c) heap.push({load[static_cast<size_t>(c)], c});
+  int32_t slot = 0;
+  for (const WorkItem& it : given) {
+    int32_t remaining = it.n_total, kb = it.kb0;
+    const int32_t first_slot = slot;
+    std::vector<std::pair<int32_t, size_t>> placed;  // (cta, index in its list)
+    while (remaining > 0) {
+      Load l = heap.top();
+      heap.pop();
+      int64_t k = std::max<int64_t>(kMinPartBlocks, target - l.first - kPartOverhead);
+      k = std::min<int64_t>(k, remaining);
+      if (remaining - k > 0 && remaining - k < kMinPartBlocks) k = remaining;  // no tiny tail
+      WorkItem part = it;
+      part.kb0 = kb;
+      part.n_total = static_cast<int32_t>(k);
+      part.part = slot++;
+      auto& dst = (*lists)[static_cast<size_t>(l.second)];
+      placed.emplace_back(l.second, dst.size());
+      dst.push_back(part);
+      l.first += k + kPartOverhead;
+      heap.push(l);
+      remaining -= static_cast<int32_t>(k);
+      kb += static_cast<int32_t>(k);
+    }
+    if (placed.size() == 1) {  // fitted whole: no partial results
+      (*lists)[static_cast<size_t>(placed[0].first)][placed[0].second].part = -1;
+      --slot;
+      continue;
+    }
+    WorkItem whole = it;
+    whole.part = first_slot;
+    whole.n_parts = static_cast<int32_t>(placed.size());
+    splits->push_back(whole);
+  }
+  int64_t makespan = 0;
+  while (!heap.empty()) {
+    makespan = std::max(makespan, heap.top().first);
+    heap.pop();
+  }
   return makespan;
 }
 
@@ -353,6 +375,7 @@ void assign_ctas(Plan* plan, int32_t ctas, bool allow_split, bool force_split) {
       const int32_t slot = 2 * static_cast<int32_t>(plan->splits.size());
       WorkItem whole = it;
       whole.part = slot;
+      whole.n_parts = 2;
       plan->splits.push_back(whole);
       WorkItem head = it, tail = it;
       head.n_total = it.n_total / 2;
@@ -375,26 +398,28 @@ void assign_ctas(Plan* plan, int32_t ctas, bool allow_split, bool force_split) {
   if (!n) return;
   std::vector<int32_t> owner;
   const int64_t lpt_span = lpt(plan->items, g, &owner);
+  std::vector<std::vector<WorkItem>> lists;
+  std::vector<WorkItem> splits;
+  int64_t span = lpt_span;
+  bool use_split = false;
   if (allow_split && !force_split && g > 1) {
-    std::vector<WorkItem> wrapped, splits;
-    std::vector<int32_t> offsets;
-    const int64_t span = wrap_around(plan->items, g, &wrapped, &offsets, &splits);
-    if (!splits.empty() && span + kSplitPenalty < lpt_span) {
-      plan->items.swap(wrapped);
-      plan->cta_offsets.swap(offsets);
-      plan->splits.swap(splits);
-      plan->makespan = span;
-      return;
-    }
+    span = tail_split(plan->items, g, owner, &lists, &splits);
+    use_split = !splits.empty() && span + kSplitPenalty < lpt_span;
   }
-  plan->makespan = lpt_span;
-  std::vector<int32_t> count(static_cast<size_t>(g), 0);
-  for (int32_t i = 0; i < n; ++i) ++count[static_cast<size_t>(owner[static_cast<size_t>(i)])];
-  for (int32_t c = 0; c < g; ++c) plan->cta_offsets[static_cast<size_t>(c) + 1] = plan->cta_offsets[static_cast<size_t>(c)] + count[static_cast<size_t>(c)];
-  std::vector<WorkItem> ordered(static_cast<size_t>(n));
-  std::vector<int32_t> at(plan->cta_offsets.begin(), plan->cta_offsets.end() - 1);
-  for (int32_t i = 0; i < n; ++i)  // stable: each CTA keeps the longest-first order
-    ordered[static_cast<size_t>(at[static_cast<size_t>(owner[static_cast<size_t>(i)])]++)] = plan->items[static_cast<size_t>(i)];
+  if (!use_split) {  // the longest-first lists, each CTA keeping the longest-first order
+    lists.assign(static_cast<size_t>(g), {});
+    for (int32_t i = 0; i < n; ++i)
+      lists[static_cast<size_t>(owner[static_cast<size_t>(i)])].push_back(plan->items[static_cast<size_t>(i)]);
+    span = lpt_span;
+  } else {
+    plan->splits.swap(splits);
+  }
+  plan->makespan = span;
+  std::vector<WorkItem> ordered;
+  for (int32_t c = 0; c < g; ++c) {
+    ordered.insert(ordered.end(), lists[static_cast<size_t>(c)].begin(), lists[static_cast<size_t>(c)].end());
+    plan->cta_offsets[static_cast<size_t>(c) + 1] = static_cast<int32_t>(ordered.size());
+  }
   plan->items.swap(ordered);
 }
 

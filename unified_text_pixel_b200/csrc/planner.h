@@ -31,9 +31,9 @@ constexpr int32_t kMaxTokens = (1 << 19) - 1;
 // kb | class << 24 with class an hgx_tile_class (FULL or PARTIAL; skipped blocks are not
 // listed).
 // Split items (part >= 0, prefix form only): the key blocks of one (query block, KV head)
-// are divided between two work items that may run on different CTAs; each writes its
+// are divided between several work items that may run on different CTAs; each writes its
 // unnormalised O, row maximum and row sum to partial-result slot `part`, and a combine
-// kernel merges the two slots into out.
+// kernel merges the item's slots into out.
 struct WorkItem {
   int32_t q0;        // packed index of the first query token
   int32_t kv0;       // packed index of the batch element's first token
@@ -45,7 +45,8 @@ struct WorkItem {
   int32_t first;     // rows before this local row are not written (cached prefix)
   int32_t kb0 = 0;   // prefix form: first key block processed
   int32_t part = -1; // -1: writes out; else its partial-result slot
-  int32_t pad[2] = {0, 0};
+  int32_t n_parts = 0;  // Plan::splits entries: number of parts (slots part .. part + n_parts - 1)
+  int32_t pad = 0;
 };
 static_assert(sizeof(WorkItem) == 48, "work item layout");
 
@@ -67,8 +68,8 @@ struct Plan {
   // [cta_offsets[c], cta_offsets[c + 1]) of `items`, longest first.
   int32_t grid = 0;
   std::vector<int32_t> cta_offsets;
-  // Split items (assign_ctas with splitting): split i wrote partial slots 2i and 2i + 1;
-  // splits[i] is the whole (query block, KV head) item with part = 2i.
+  // Split items (assign_ctas with splitting): splits[i] is the whole (query block, KV head)
+  // item whose parts wrote the partial slots part .. part + n_parts - 1.
   std::vector<WorkItem> splits;
   int64_t makespan = 0;  // largest CTA load of the assignment, in key blocks + overheads
 };
@@ -99,11 +100,10 @@ hgx_status check_first_rows(int32_t batch, const int32_t* cu_seqlens, const hgx_
 // overhead), reorders the items so that every CTA's list is contiguous, and sets grid,
 // cta_offsets and makespan. grid = min(ctas, number of items).
 //
-// With allow_split, a second schedule is tried: the wrap-around rule for preemptive
-// scheduling (McNaughton) -- the CTAs are filled one after the other up to a common bound,
-// and a prefix-form item that straddles a CTA's bound is split by key blocks into two
-// items, the first finishing that CTA's list and the second opening the next one. It
-// replaces the first schedule when its makespan plus kSplitPenalty is smaller.
+// With allow_split, a second schedule is tried: the CTAs loaded above the mean give back
+// their last (smallest) items, whose key blocks are handed out in parts to the least-loaded
+// CTAs (tail_split in planner.cpp). It replaces the first schedule when its makespan plus
+// kSplitPenalty is smaller.
 constexpr int64_t kItemOverhead = 2;   // loading Q and writing O: about two key blocks
 constexpr int64_t kSplitPenalty = 3;   // the combine launch, in key blocks
 // force_split (a test hook that exercises the split path on any input): every prefix-form

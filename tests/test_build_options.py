@@ -2,7 +2,8 @@
 
 The default build is covered by every other test; these are the alternatives kept in the
 source (two softmax warps per row, P in four or one parts, polynomial exp2 for part of
-the scores, direct epilogue stores, no split items). Each is compiled to an object file with nvcc, in parallel.
+the scores, direct epilogue stores, no split items, the first prologue layout, a 64-thread
+prologue block). Each is compiled to an object file with nvcc, in parallel.
 """
 import os
 import shutil
@@ -22,6 +23,8 @@ OPTIONS = {
     "polynomial_exp2": ["-DHGX_EXP_POLY_MASK=0x0101"],
     "no_split_items": ["-DHGX_SPLIT_KV=0"],
     "direct_epilogue_stores": ["-DHGX_EPI_TMA=0"],
+    "first_prologue_layout": ["-DHGX_PRO_V2=0"],
+    "prologue_64_threads": ["-DHGX_PRO_V2_THREADS=64"],
 }
 
 
@@ -32,7 +35,8 @@ def test_attention_options_compile():
     with tempfile.TemporaryDirectory() as tmp:
         procs = {}
         for name, flags in OPTIONS.items():
-            target = os.path.join(CSRC, "api.cu") if "SPLIT_KV" in flags[0] else src
+            target = (os.path.join(CSRC, "api.cu") if "SPLIT_KV" in flags[0] else
+                      os.path.join(CSRC, "prologue.cu") if "PRO_" in flags[0] else src)
             cmd = [nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17",
                    "-I", CSRC, *flags, "-c", target, "-o", os.path.join(tmp, name + ".o")]
             procs[name] = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT)

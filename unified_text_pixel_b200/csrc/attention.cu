@@ -762,12 +762,14 @@ __global__ void __launch_bounds__(256) combine_kernel(const WorkItem* __restrict
   if (!(tok - it.kv0 < it.len && tok - it.kv0 >= it.first)) return;
   auto prow = [&](int i) { return (static_cast<size_t>(it.part + i) * 2 + x) * 128 + row; };
   float m = -INFINITY;
+#pragma unroll 4
   for (int i = 0; i < it.n_parts; ++i) {
     const float2 ml = pml[prow(i)];
     if (ml.y > 0.f) m = fmaxf(m, ml.x);  // finite: every written row sees at least itself
   }
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float den = 0.f;
+#pragma unroll 4
   for (int i = 0; i < it.n_parts; ++i) {
     const float2 ml = pml[prow(i)];
     if (!(ml.y > 0.f)) continue;  // the row saw no key of this part

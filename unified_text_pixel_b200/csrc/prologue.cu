@@ -6,15 +6,11 @@
 // the 1D RoPE definition in "HunyuanImage 3.0 Technical Report" (paper-graph-ui summary),
 // section 3.4, "Generalized 2D Rotary Position Embedding (RoPE)".
 //
-// Layout: one block handles kTok tokens and all 40 heads (32 q + 8 k) of each (1 token,
-// 64 threads: many small blocks keep loads in flight while others compute). A head's
-// 128 bf16 (256 B) is read by a half-warp as 16-byte loads, so a warp reads 512
-// contiguous bytes; lanes j and j + 8 of a half-warp hold the partners (k, k + 64) of a
-// rotation and swap values with one shuffle. Angles are computed once per (token, k) in
-// fp64 (positions reach ~10^4 rad, far outside the range where a float angle keeps
-// precision) and shared by all 40 heads through shared memory; they are computed while
-// the thread's loads (all issued first, 160 bytes per thread) are in flight. HBM-bound:
-// every byte of q and k is read once and written once.
+// HBM-bound: every byte of q and k is read once and written once. The default kernel
+// (prologue_v2_kernel, described at its definition) gives each thread both members of its
+// rotation pairs and reduces the angles exactly in fp32; the first layout (prologue_kernel,
+// HGX_PRO_V2=0: a half-warp per head, partners exchanged by shuffles, fp64 angles) is kept
+// for comparison.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -145,12 +141,130 @@ __global__ void __launch_bounds__(kThreads, kProMinBlocks) prologue_kernel(
   }
 }
 
+// ----------------------------------------------------------------------------------------
+// Second layout (HGX_PRO_V2, default): a thread holds both members of its rotation pairs --
+// features 8j .. 8j+7 and 64+8j .. 64+8j+7 of a head (two 16-byte loads) -- so the rotation
+// needs no shuffle; eight threads cover a head (the sum of squares is reduced over them with
+// three shuffles) and the 64 threads of a block five heads each. The (cos, sin) table is
+// stored transposed, entry (e, j) for frequency 8j + e, so that the eight threads of a head
+// read 64 consecutive bytes (no bank conflicts). Angles are reduced in fp32 without loss:
+// the position is an integer below 2^24, u = inv_freq / 2pi is split into u_hi + u_lo
+// (floats), pos * u_hi is exact as hi + err (an FMA gives the rounding error), and the
+// fraction of a turn r = (hi - rint(hi)) + (err + pos * u_lo) carries an error near 2^-25;
+// sincospif(2r) gives cos and sin of 2 pi r. Positions of 2^24 or more take the fp64 sincos.
+struct RopeTurns {
+  float u_hi[64];
+  float u_lo[64];
+  double inv_freq[64];
+  uint8_t axis[64];
+};
+
+#ifndef HGX_PRO_V2
+#define HGX_PRO_V2 1
+#endif
+#ifndef HGX_PRO_V2_THREADS
+#define HGX_PRO_V2_THREADS 160
+#endif
+constexpr int kV2Threads = HGX_PRO_V2_THREADS;  // 8 per head in flight
+constexpr int kV2Units = kHeads * 8 / kV2Threads;  // heads per thread
+static_assert(kV2Threads % 64 == 0 || kV2Threads == 160 || kV2Threads == 320, "block shape");
+static_assert(kHeads * 8 % kV2Threads == 0, "heads must split evenly over the threads");
+// resident blocks per SM the register allocation must allow (no spills at these shapes)
+constexpr int kV2MinBlocks = kV2Threads == 320 ? 6 : kV2Threads == 160 ? 8 : 10;
+
+__global__ void __launch_bounds__(kV2Threads, kV2MinBlocks) prologue_v2_kernel(
+    __nv_bfloat16* __restrict__ q, __nv_bfloat16* __restrict__ k,
+    const int32_t* __restrict__ pos, const __nv_bfloat16* __restrict__ wq,
+    const __nv_bfloat16* __restrict__ wk, int32_t T, float eps, const __grid_constant__ RopeTurns tab) {
+  __shared__ float2 cs[8][8];  // (cos, sin) of frequency 8j + e at [e][j]
+  const int t = blockIdx.x;
+  const int j = threadIdx.x & 7;   // pair chunk: features 8j.. and 64+8j..
+  const int u0 = threadIdx.x >> 3; // first head of this thread (kV2Threads / 8 in flight)
+  // 1. the angle of frequency f = threadIdx.x (fp32 fast path: a few dozen instructions)
+  if (threadIdx.x < 64) {
+    const int f = threadIdx.x;
+    const int32_t pv = pos[3 * t + tab.axis[f]];
+    float c, sn;
+    if (pv > -(1 << 24) && pv < (1 << 24)) {
+      const float pf = static_cast<float>(pv);
+      const float h = pf * tab.u_hi[f];
+      const float err = fmaf(pf, tab.u_hi[f], -h);
+      const float r = (h - rintf(h)) + fmaf(pf, tab.u_lo[f], err);
+      sincospif(2.f * r, &sn, &c);
+    } else {
+      double sd, cd;
+      sincos(static_cast<double>(pv) * tab.inv_freq[f], &sd, &cd);
+      c = static_cast<float>(cd);
+      sn = static_cast<float>(sd);
+    }
+    cs[f & 7][f >> 3] = make_float2(c, sn);
+  }
+  // 2. the loads: kV2Units heads x 2 chunks of 16 bytes, all in flight before any is used
+  uint4 lo[kV2Units], hi[kV2Units];
+#pragma unroll
+  for (int n = 0; n < kV2Units; ++n) {
+    const int hh = u0 + (kV2Threads / 8) * n;
+    const __nv_bfloat16* base = hh < 32 ? q + (static_cast<size_t>(t) * 32 + hh) * 128
+                                        : k + (static_cast<size_t>(t) * 8 + (hh - 32)) * 128;
+    lo[n] = *reinterpret_cast<const uint4*>(base + 8 * j);
+    hi[n] = *reinterpret_cast<const uint4*>(base + 64 + 8 * j);
+  }
+  __syncthreads();
+  float2 cj[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) cj[e] = cs[e][j];
+  // 3. normalise, rotate, store
+#pragma unroll
+  for (int n = 0; n < kV2Units; ++n) {
+    const int hh = u0 + (kV2Threads / 8) * n;
+    float a[8], b[8];
+    unpack8(lo[n], a);
+    unpack8(hi[n], b);
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ss = fmaf(a[e], a[e], fmaf(b[e], b[e], ss));
+#pragma unroll
+    for (int off = 4; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    const float r = rsqrtf(ss * (1.f / 128.f) + eps);
+    // norm weights of this thread's 16 features (L1-resident after the first token)
+    const __nv_bfloat16* wsrc = hh < 32 ? wq : wk;
+    float wa[8], wb[8];
+    unpack8(__ldg(reinterpret_cast<const uint4*>(wsrc + 8 * j)), wa);
+    unpack8(__ldg(reinterpret_cast<const uint4*>(wsrc + 64 + 8 * j)), wb);
+    float oa[8], ob[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float ya = a[e] * r * wa[e], yb = b[e] * r * wb[e];
+      oa[e] = fmaf(ya, cj[e].x, -yb * cj[e].y);
+      ob[e] = fmaf(yb, cj[e].x, ya * cj[e].y);
+    }
+    __nv_bfloat16* base = hh < 32 ? q + (static_cast<size_t>(t) * 32 + hh) * 128
+                                  : k + (static_cast<size_t>(t) * 8 + (hh - 32)) * 128;
+    *reinterpret_cast<uint4*>(base + 8 * j) = pack8(oa);
+    *reinterpret_cast<uint4*>(base + 64 + 8 * j) = pack8(ob);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_prologue(cudaStream_t stream, void* q, void* k, const int32_t* pos,
                             const void* wq, const void* wk, int32_t T, float eps,
                             const RopeTables& tab) {
   if (T <= 0) return cudaSuccess;
+  if constexpr (HGX_PRO_V2 != 0) {
+    RopeTurns turns{};
+    for (int f = 0; f < 64; ++f) {
+      const double u = tab.inv_freq[f] / (2.0 * 3.14159265358979323846);
+      turns.u_hi[f] = static_cast<float>(u);
+      turns.u_lo[f] = static_cast<float>(u - static_cast<double>(turns.u_hi[f]));
+      turns.inv_freq[f] = tab.inv_freq[f];
+      turns.axis[f] = tab.axis[f];
+    }
+    prologue_v2_kernel<<<T, kV2Threads, 0, stream>>>(
+        static_cast<__nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(k), pos,
+        static_cast<const __nv_bfloat16*>(wq), static_cast<const __nv_bfloat16*>(wk), T, eps, turns);
+    return cudaGetLastError();
+  }
   const int grid = (T + kTok - 1) / kTok;
   prologue_kernel<<<grid, kThreads, 0, stream>>>(
       static_cast<__nv_bfloat16*>(q), static_cast<__nv_bfloat16*>(k), pos,

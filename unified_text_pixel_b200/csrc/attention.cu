@@ -80,6 +80,12 @@ constexpr int kStages = HGX_KV_STAGES;        // K/V ring slots
 // that the PV MMAs of the first parts overlap the exponentials of the later ones
 constexpr int kPParts = HGX_P_PARTS;
 static_assert(kPParts == 1 || kPParts == 2 || kPParts == 4, "P parts");
+#ifndef HGX_SPLIT_LD
+#define HGX_SPLIT_LD 1
+#endif
+// 1: in fully visible blocks the softmax loads S in two halves and takes the maximum of the
+// first half while the second half is loading
+constexpr bool kSplitLd = HGX_SPLIT_LD != 0 && kSplit == 1;
 constexpr uint32_t kTileBytes = 32768;        // 128 rows x 128 bf16
 constexpr uint32_t kHalfBytes = 16384;        // 128 rows x 64 bf16 (one 128-byte swizzle span)
 constexpr uint32_t kQBytes = 2 * kTileBytes;  // both Q tiles of an item
@@ -508,10 +514,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         // (with two halves an aborted wait still loads: tensor memory is always readable,
         // and the tile decides together at the exchange below)
         uint32_t sr[kCols / 32][32];
+        float s[kCols];
+        float mx;
+        // row max: independent chains of 16 scores (three-input max), then a tree; a single
+        // long chain would expose its whole latency
+        auto chain16 = [&](int i) {
+          const float* c16 = s + 16 * i;
+          float m = fmax3(c16[0], c16[1], c16[2]);
+#pragma unroll
+          for (int e = 3; e < 15; e += 2) m = fmax3(m, c16[e], c16[e + 1]);
+          return fmaxf(m, c16[15]);
+        };
+        if (kSplitLd && full) {
+          // a fully visible block: the second half of the row loads while the maximum of
+          // the first half is computed
+          tmem_ld32(tS, sr[0]);
+          tmem_ld32(tS + 32, sr[1]);
+          tmem_wait_ld();
+          tmem_ld32(tS + 64, sr[2]);
+          tmem_ld32(tS + 96, sr[3]);
+#pragma unroll
+          for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) s[32 * ch + e] = __uint_as_float(sr[ch][e]);
+          const float ma = fmaxf(fmaxf(chain16(0), chain16(1)), fmaxf(chain16(2), chain16(3)));
+          tmem_wait_ld();
+#pragma unroll
+          for (int ch = 2; ch < 4; ++ch)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) s[32 * ch + e] = __uint_as_float(sr[ch][e]);
+          mx = fmaxf(ma, fmaxf(fmaxf(chain16(4), chain16(5)), fmaxf(chain16(6), chain16(7))));
+        } else {
 #pragma unroll
         for (int ch = 0; ch < kCols / 32; ++ch) tmem_ld32(tS + 32 * ch, sr[ch]);
         tmem_wait_ld();
-        float s[kCols];
 #pragma unroll
         for (int ch = 0; ch < kCols / 32; ++ch)
 #pragma unroll
@@ -538,20 +574,13 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (e >= nvis) s[e] = -INFINITY;
           }
         }
-        // row max: independent chains of 16 scores (three-input max), then a tree; a single
-        // long chain would expose its whole latency
         float m8[kCols / 16];
 #pragma unroll
-        for (int i = 0; i < kCols / 16; ++i) {
-          const float* c16 = s + 16 * i;
-          float m = fmax3(c16[0], c16[1], c16[2]);
-#pragma unroll
-          for (int e = 3; e < 15; e += 2) m = fmax3(m, c16[e], c16[e + 1]);
-          m8[i] = fmaxf(m, c16[15]);
-        }
-        float mx = m8[0];
+        for (int i = 0; i < kCols / 16; ++i) m8[i] = chain16(i);
+        mx = m8[0];
 #pragma unroll
         for (int i = 1; i < kCols / 16; ++i) mx = fmaxf(mx, m8[i]);
+        }
         if constexpr (kSplit == 2) {
           // exchange with the other half of the row; the barrier also decides, for the
           // whole tile, whether every wait succeeded

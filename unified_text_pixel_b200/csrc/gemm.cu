@@ -35,6 +35,10 @@ using namespace waits;
 #define HGX_GEMM_L2_HINTS 1
 #endif
 constexpr bool kL2Hints = HGX_GEMM_L2_HINTS != 0;  // L2 cache policies on the operand loads
+#ifndef HGX_GEMM_A_FIRST
+#define HGX_GEMM_A_FIRST 1
+#endif
+constexpr bool kAFirst = HGX_GEMM_A_FIRST != 0;
 constexpr int kThreads = 192;
 constexpr int BM = 128, BN = 256, BK = 64, kStages = 4;
 constexpr uint32_t kABytes = BM * BK * 2;  // 16 KB
@@ -82,12 +86,26 @@ __device__ __forceinline__ void norm_rope_row(float (&x)[128], const float* w, c
   }
 }
 
-__device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const float (&x)[128]) {
+#ifndef HGX_GEMM_STORE_FIRST
+#define HGX_GEMM_STORE_FIRST 1
+#endif
+// 1: the epilogue's stores carry an L2 evict-first policy (the outputs are read by the next
+// kernel, not by this one), so that they do not push the weights out of L2
+constexpr bool kStoreFirst = HGX_GEMM_STORE_FIRST != 0;
+
+__device__ __forceinline__ void store_row_bf16(__nv_bfloat16* dst, const float (&x)[128], uint64_t policy) {
   uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-  for (int e = 0; e < 16; ++e)
-    d4[e] = make_uint4(pack_bf16x2(x[8 * e], x[8 * e + 1]), pack_bf16x2(x[8 * e + 2], x[8 * e + 3]),
-                       pack_bf16x2(x[8 * e + 4], x[8 * e + 5]), pack_bf16x2(x[8 * e + 6], x[8 * e + 7]));
+  for (int e = 0; e < 16; ++e) {
+    const uint4 v = make_uint4(pack_bf16x2(x[8 * e], x[8 * e + 1]), pack_bf16x2(x[8 * e + 2], x[8 * e + 3]),
+                               pack_bf16x2(x[8 * e + 4], x[8 * e + 5]), pack_bf16x2(x[8 * e + 6], x[8 * e + 7]));
+    if constexpr (kStoreFirst)
+      asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(d4 + e), "r"(v.x),
+                   "r"(v.y), "r"(v.z), "r"(v.w), "l"(policy)
+                   : "memory");
+    else
+      d4[e] = v;
+  }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -152,10 +170,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(full, kStageBytes);
           const uint32_t sa = base + slot * kStageBytes;
           if constexpr (kL2Hints) {
-            // the weights (B) are read again by every row block: keep them in L2; the
-            // activations (A) are read by the column tiles of their row block at about the
-            // same time and then never again
-            tma_load_2d_hint(sa, &tmap_a, full, kb * BK, m0, pol_a);
+            // the weights (B) are read again by every row block: keep them in L2 (evict
+            // last); the activations (A) are read by the column tiles of their row block at
+            // about the same time (evict first when HGX_GEMM_A_FIRST, else the default)
+            if constexpr (kAFirst)
+              tma_load_2d_hint(sa, &tmap_a, full, kb * BK, m0, pol_a);
+            else
+              tma_load_2d(sa, &tmap_a, full, kb * BK, m0);
             tma_load_2d_hint(sa + kABytes, &tmap_b, full, kb * BK, n0, pol_b);
           } else {
             tma_load_2d(sa, &tmap_a, full, kb * BK, m0);
@@ -203,6 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------------ epilogue
     const int quarter = warp & 3;
+    const uint64_t store_pol = l2_policy_evict_first();
     const int row = quarter * 32 + lane;
     const uint32_t lane_bits = static_cast<uint32_t>(quarter * 32) << 16;
     int lt = 0;
@@ -229,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!valid) continue;
         const int col = n0 + 128 * h;
         if (p.mode == 0) {
-          store_row_bf16(static_cast<__nv_bfloat16*>(p.c) + static_cast<size_t>(token) * p.N + col, x);
+          store_row_bf16(static_cast<__nv_bfloat16*>(p.c) + static_cast<size_t>(token) * p.N + col, x, store_pol);
         } else {
           const int head = col / 128;  // 0..31 q, 32..39 k, 40..47 v
           __nv_bfloat16* dst;
@@ -242,7 +264,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             dst = static_cast<__nv_bfloat16*>(p.v) + (static_cast<size_t>(token) * 8 + (head - 40)) * 128;
           }
-          store_row_bf16(dst, x);
+          store_row_bf16(dst, x, store_pol);
         }
       }
       tc_fence_before();

@@ -325,6 +325,7 @@ hgx_status run_attention(hgx_attn_handle* h, cudaStream_t stream, const void* q,
   p.partial_ml = slots ? reinterpret_cast<float2*>(static_cast<float*>(h->d_partial) +
                                                    slots * hgx::kPartialSlotFloats)
                        : nullptr;
+
   p.scale_log2 = h->scale * 1.4426950408889634f;
   p.flags = h->flags;
   p.err = h->d_err;

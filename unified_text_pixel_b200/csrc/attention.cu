@@ -777,8 +777,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// One warp per row of a split item: lane i merges features 4i .. 4i + 3 over the item's
-// n_parts partial results, out = sum_p O_p 2^(M_p - M) / sum_p l_p 2^(M_p - M), M = max M_p.
+// One warp per row of a split item: out = sum_p O_p 2^(M_p - M) / sum_p l_p 2^(M_p - M),
+// M = max M_p over the parts the row saw keys in. Lane i first reads the (M, l) of parts i,
+// i + 32, ... (all at once), the warp reduces the maximum and the denominator with
+// shuffles, and then every lane accumulates features 4i .. 4i + 3 over the parts with
+// independent loads (a part whose row saw no key has O = 0 and weight 0).
 __global__ void __launch_bounds__(256) combine_kernel(const WorkItem* __restrict__ splits, int32_t n_splits,
                                                       const float* __restrict__ po,
                                                       const float2* __restrict__ pml, __nv_bfloat16* out) {
@@ -790,25 +793,31 @@ __global__ void __launch_bounds__(256) combine_kernel(const WorkItem* __restrict
   const int32_t tok = it.q0 + 32 * x + (row >> 2);
   if (!(tok - it.kv0 < it.len && tok - it.kv0 >= it.first)) return;
   auto prow = [&](int i) { return (static_cast<size_t>(it.part + i) * 2 + x) * 128 + row; };
+  const int np = it.n_parts;
   float m = -INFINITY;
-#pragma unroll 4
-  for (int i = 0; i < it.n_parts; ++i) {
+  for (int i = lane; i < np; i += 32) {
     const float2 ml = pml[prow(i)];
     if (ml.y > 0.f) m = fmaxf(m, ml.x);  // finite: every written row sees at least itself
   }
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
   float den = 0.f;
-#pragma unroll 4
-  for (int i = 0; i < it.n_parts; ++i) {
+  for (int i = lane; i < np; i += 32) {
     const float2 ml = pml[prow(i)];
-    if (!(ml.y > 0.f)) continue;  // the row saw no key of this part
-    const float wgt = exp2f(ml.x - m);
+    if (ml.y > 0.f) den = fmaf(ml.y, exp2f(ml.x - m), den);
+  }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+  for (int i = 0; i < np; ++i) {
+    const float2 ml = pml[prow(i)];  // the same address for all lanes: one broadcast load
+    const float wgt = ml.y > 0.f ? exp2f(ml.x - m) : 0.f;
     const float4 o = reinterpret_cast<const float4*>(po + prow(i) * 128)[lane];
     acc.x = fmaf(o.x, wgt, acc.x);
     acc.y = fmaf(o.y, wgt, acc.y);
     acc.z = fmaf(o.z, wgt, acc.z);
     acc.w = fmaf(o.w, wgt, acc.w);
-    den = fmaf(ml.y, wgt, den);
   }
   const float inv = 1.f / den;
   const uint32_t lo = pack_bf16x2(acc.x * inv, acc.y * inv);

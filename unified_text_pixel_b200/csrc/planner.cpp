@@ -347,6 +347,11 @@ int64_t tail_split(const std::vector<WorkItem>& items, int32_t g, const std::vec
       --slot;
       continue;
     }
+    for (const auto& pl : placed) {  // every part knows its item's slots (merge in the kernel)
+      WorkItem& part = (*lists)[static_cast<size_t>(pl.first)][pl.second];
+      part.n_parts = static_cast<int32_t>(placed.size());
+      part.pad = first_slot;
+    }
     WorkItem whole = it;
     whole.part = first_slot;
     whole.n_parts = static_cast<int32_t>(placed.size());
@@ -383,6 +388,8 @@ void assign_ctas(Plan* plan, int32_t ctas, bool allow_split, bool force_split) {
       tail.kb0 = it.kb0 + head.n_total;
       tail.n_total = it.n_total - head.n_total;
       tail.part = slot + 1;
+      head.n_parts = tail.n_parts = 2;
+      head.pad = tail.pad = slot;
       halves.push_back(head);
       halves.push_back(tail);
     }

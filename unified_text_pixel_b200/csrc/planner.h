@@ -45,8 +45,8 @@ struct WorkItem {
   int32_t first;     // rows before this local row are not written (cached prefix)
   int32_t kb0 = 0;   // prefix form: first key block processed
   int32_t part = -1; // -1: writes out; else its partial-result slot
-  int32_t n_parts = 0;  // Plan::splits entries: number of parts (slots part .. part + n_parts - 1)
-  int32_t pad = 0;
+  int32_t n_parts = 0;  // split items: number of parts of the whole item
+  int32_t pad = 0;      // parts of split items: the whole item's first slot (Plan::splits: part)
 };
 static_assert(sizeof(WorkItem) == 48, "work item layout");
 

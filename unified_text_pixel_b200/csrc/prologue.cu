@@ -180,7 +180,18 @@ __global__ void __launch_bounds__(kV2Threads, kV2MinBlocks) prologue_v2_kernel(
   const int t = blockIdx.x;
   const int j = threadIdx.x & 7;   // pair chunk: features 8j.. and 64+8j..
   const int u0 = threadIdx.x >> 3; // first head of this thread (kV2Threads / 8 in flight)
-  // 1. the angle of frequency f = threadIdx.x (fp32 fast path: a few dozen instructions)
+  // 1. the loads: kV2Units heads x 2 chunks of 16 bytes, all in flight before any is used (and
+  // before the angles, whose arithmetic then overlaps them)
+  uint4 lo[kV2Units], hi[kV2Units];
+#pragma unroll
+  for (int n = 0; n < kV2Units; ++n) {
+    const int hh = u0 + (kV2Threads / 8) * n;
+    const __nv_bfloat16* base = hh < 32 ? q + (static_cast<size_t>(t) * 32 + hh) * 128
+                                        : k + (static_cast<size_t>(t) * 8 + (hh - 32)) * 128;
+    lo[n] = *reinterpret_cast<const uint4*>(base + 8 * j);
+    hi[n] = *reinterpret_cast<const uint4*>(base + 64 + 8 * j);
+  }
+  // 2. the angle of frequency f = threadIdx.x (fp32 fast path: a few dozen instructions)
   if (threadIdx.x < 64) {
     const int f = threadIdx.x;
     const int32_t pv = pos[3 * t + tab.axis[f]];
@@ -198,16 +209,6 @@ __global__ void __launch_bounds__(kV2Threads, kV2MinBlocks) prologue_v2_kernel(
       sn = static_cast<float>(sd);
     }
     cs[f & 7][f >> 3] = make_float2(c, sn);
-  }
-  // 2. the loads: kV2Units heads x 2 chunks of 16 bytes, all in flight before any is used
-  uint4 lo[kV2Units], hi[kV2Units];
-#pragma unroll
-  for (int n = 0; n < kV2Units; ++n) {
-    const int hh = u0 + (kV2Threads / 8) * n;
-    const __nv_bfloat16* base = hh < 32 ? q + (static_cast<size_t>(t) * 32 + hh) * 128
-                                        : k + (static_cast<size_t>(t) * 8 + (hh - 32)) * 128;
-    lo[n] = *reinterpret_cast<const uint4*>(base + 8 * j);
-    hi[n] = *reinterpret_cast<const uint4*>(base + 64 + 8 * j);
   }
   __syncthreads();
   float2 cj[8];

@@ -281,12 +281,20 @@ L2_FLUSH_BYTES = 256 << 20  # twice the 126 MB L2
 
 def per_workload_timings(H, a, peaks, iters=10, names=PER_WORKLOAD):
     """Event-timed prologue and attention launches of every workload, each launch preceded by
-    a write of a buffer twice the size of L2 (outside the timed launch), on pristine q/k
-    restored before every prologue. Returns {name: figures}."""
+    an L2 flush outside the timed launch (a write of a buffer twice the size of L2, then a
+    read of another one of that size, so that the launch starts with none of its inputs in
+    L2 and with no dirty lines there: after the write alone, the timed kernel would also pay
+    for writing the flush buffer back to HBM), on pristine q/k restored before every
+    prologue. Returns {name: figures}."""
     import torch
 
     stream = torch.cuda.current_stream()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    sweep = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+
+    def cold_l2():
+        flush.zero_()
+        sweep.sum()
     res = {}
     for name in names:
         w = _workload(name)
@@ -304,11 +312,11 @@ def per_workload_timings(H, a, peaks, iters=10, names=PER_WORKLOAD):
             for n in d:
                 d[n].copy_(pristine[n])
             ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-            flush.zero_()
+            cold_l2()
             ev[0].record(stream)
             a.prologue(d["q"], d["k"], pos, wq, wk, stream=stream)
             ev[1].record(stream)
-            flush.zero_()
+            cold_l2()
             ev[2].record(stream)
             a.attention(d["q"], d["k"], v, out, cu, segs, cu_segs, stream=stream)
             ev[3].record(stream)
@@ -527,6 +535,9 @@ def run_gpu(args):
     if not args.no_per_workload and not first_rows:
         _log("per-workload kernel timings")
         line["per_workload"] = per_workload_timings(H, a, peaks)
+        line["per_workload_method"] = ("each kernel event-timed alone, median of 10 launches; before each launch "
+                                       "the L2 is flushed by writing 256 MB and then reading 256 MB (cold and "
+                                       "clean); q/k restored before each prologue")
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         _log("cpu baseline (oracle)")
         v, rows, secs, threads = cpu_oracle_sample(w, budget_s=args.cpu_seconds)

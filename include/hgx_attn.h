@@ -292,7 +292,7 @@ hgx_status hgx_attn_set_debug(hgx_attn_handle* h, uint32_t flags, uint64_t wait_
  * the limits: at most HGX_NOALLOC_MAX_TOKENS packed tokens and HGX_NOALLOC_MAX_BATCH batch
  * elements, and no gen_image segments; other requests return HGX_ERR_UNSUPPORTED before
  * any device work. Work items are assigned to the persistent CTAs as in hgx_attn_forward
- * (longest first, each to the least-loaded CTA).
+ * (largest planned cost first, each to the least-loaded CTA).
  *
  * Arguments are those of hgx_attn_forward with the config in place of a handle (validated
  * on every call), plus `synchronize`: when nonzero the call waits for the stream and returns

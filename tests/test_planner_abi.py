@@ -391,15 +391,22 @@ def test_split_schedule_covers_every_key_block_once(case, split_test):
     # execution order: CTAs in order, every CTA's items contiguous
     assert (np.diff(s[:, 0]) >= 0).all()
     used = int(s[:, 0].max()) + 1
-    lpt = _lpt_makespan([int(r[4]) + 2 for r in base], ctas)
+
+    # the planner's cost model, in tenths of a fully visible key block: 10 per fully visible
+    # block, 13 per block that needs the mask compare, + 12 per item, + 30 per part of a split
+    # item (prefix-form items: blocks below n_full are fully visible)
+    def cost(rows):
+        nf = np.clip(rows[:, 6] - rows[:, 3], 0, rows[:, 4])
+        return 10 * nf + 13 * (rows[:, 4] - nf) + np.where(rows[:, 5] >= 0, 30, 12)
+
+    has_lists = (base[:, 7] >= 0).any()  # list-form items: their blocks' classes are not in the rows
+    lpt = _lpt_makespan([int(x) for x in cost(base)], ctas)
     if case == "c2" and not split_test:
         assert len(slots) > 0
     if split_test:  # the test hook splits every prefix-form item of two or more key blocks
         for key, (n, _, list_off) in whole.items():
             assert len(groups[key]) == (2 if list_off < 0 and n >= 2 else 1), key
-    else:
-        # the planner's cost model: key blocks + 2 per item, + 3 per part of a split item;
+    elif not has_lists:
         # a split schedule is taken only when it beats longest-first by more than 3 blocks
-        cost = s[:, 4] + np.where(s[:, 5] >= 0, 3, 2)
-        span = np.bincount(s[:, 0], weights=cost, minlength=used).max()
-        assert (span + 3 < lpt) if slots else (span == lpt)
+        span = np.bincount(s[:, 0], weights=cost(s), minlength=used).max()
+        assert (span + 30 < lpt) if slots else (span == lpt)

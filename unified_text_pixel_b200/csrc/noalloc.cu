@@ -27,7 +27,7 @@
 // then -- which is why a call on a stream that is being captured is refused.
 //
 // Work assignment: as in the handle path, every persistent CTA gets a contiguous list of
-// items, each item (longest first) going to the least-loaded CTA; the heap of CTA loads
+// items, each item (largest planned cost first) going to the least-loaded CTA; the heap of CTA loads
 // lives in a fixed static array.
 //
 // The paper has no counterpart to this entry point; it exists for the callers above.
@@ -64,7 +64,8 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 static int32_t s_lim[kMaxTokens];
 static hgx::WorkItem s_unsorted[kMaxItems];
 static hgx::WorkItem s_items[kMaxItems];
-static int32_t s_bucket[kMaxKeyBlocks + 2];
+constexpr int64_t kMaxCost = hgx::planned_cost_bound(kMaxKeyBlocks);
+static int32_t s_bucket[kMaxCost + 2];
 static hgx::WorkItem s_assigned[kMaxItems];
 static int32_t s_owner[kMaxItems];
 static int32_t s_cta_offsets[kMaxCtas + 1];
@@ -183,7 +184,7 @@ void heap_sift_down(int32_t n) {
 }
 
 // Longest-processing-time assignment of the n sorted items of s_items to `grid` CTAs
-// (cost of an item: its key blocks plus 2 for loading Q and writing O). Fills
+// (cost of an item: hgx::planned_cost, as in the handle path). Fills
 // s_cta_offsets[0..grid] and reorders the items into s_assigned so that every CTA's list is
 // contiguous and keeps the longest-first order.
 void assign(int32_t n, int32_t grid) {
@@ -196,7 +197,7 @@ void assign(int32_t n, int32_t grid) {
     const int32_t c = s_heap_cta[0];
     s_owner[i] = c;
     ++s_cta_offsets[c + 1];
-    s_heap_load[0] += s_items[i].n_total + 2;
+    s_heap_load[0] += hgx::planned_cost(s_items[i], nullptr);
     heap_sift_down(grid);
   }
   for (int32_t c = 0; c < grid; ++c) s_cta_offsets[c + 1] += s_cta_offsets[c];
@@ -238,7 +239,7 @@ hgx_status plan(int32_t batch, const int32_t* cu, const hgx_segment* segs, const
     }
     if (at != L) return HGX_ERR_INVALID_ARG;
   }
-  // work items, then a stable counting sort by key-block count, longest first
+  // work items, then a stable counting sort by planned cost, largest first
   int32_t n = 0;
   for (int32_t b = 0; b < batch; ++b) {
     const int32_t base = cu[b], L = cu[b + 1] - cu[b];
@@ -263,9 +264,10 @@ hgx_status plan(int32_t batch, const int32_t* cu, const hgx_segment* segs, const
     }
   }
   std::memset(s_bucket, 0, sizeof(s_bucket));
-  for (int32_t i = 0; i < n; ++i) ++s_bucket[kMaxKeyBlocks - s_unsorted[i].n_total + 1];
-  for (int32_t k = 1; k < kMaxKeyBlocks + 2; ++k) s_bucket[k] += s_bucket[k - 1];
-  for (int32_t i = 0; i < n; ++i) s_items[s_bucket[kMaxKeyBlocks - s_unsorted[i].n_total]++] = s_unsorted[i];
+  for (int32_t i = 0; i < n; ++i) ++s_bucket[kMaxCost - hgx::planned_cost(s_unsorted[i], nullptr) + 1];
+  for (int64_t k = 1; k < kMaxCost + 2; ++k) s_bucket[k] += s_bucket[k - 1];
+  for (int32_t i = 0; i < n; ++i)
+    s_items[s_bucket[kMaxCost - hgx::planned_cost(s_unsorted[i], nullptr)]++] = s_unsorted[i];
   *T_out = T;
   *n_items = n;
   return HGX_OK;

@@ -265,11 +265,33 @@ hgx_status build_plan(int32_t batch, const int32_t* cu_seqlens, const hgx_segmen
 
 namespace {
 
-int64_t item_cost(const WorkItem& it) { return it.n_total + kItemOverhead; }
+// Cost of a work item in the schedule, in tenths of a fully visible key block: the kernel's
+// cycles per CTA fit a fully visible block at ~3060 cycles, a block that runs the per-score
+// mask compare (PARTIAL) at ~3900 and an item's own overhead (Q load, pipeline fill,
+// epilogue) at ~2100-3600 (B200, per-CTA clock64 counts on the edit step and the CFG pairs).
+constexpr int64_t kFullCost = 10, kPartialCost = 13;
+constexpr int64_t kPartOverhead = 30;  // an extra item's Q load, pipeline fill and epilogue, plus its share of the combine
+constexpr int32_t kMinPartBlocks = 2;
 
-// Longest processing time first; items are sorted longest first. Returns the owner of
+// kblocks: the plan's key-block lists (entries of list-form items carry their class)
+int64_t block_cost(const WorkItem& it, const uint32_t* kblocks) {
+  int64_t nf = 0;
+  if (it.list_off >= 0) {
+    for (int32_t j = 0; j < it.n_total; ++j)
+      nf += (kblocks[it.list_off + j] >> kListClassShift) == HGX_TILE_FULL;
+  } else {
+    nf = std::min<int64_t>(std::max<int64_t>(it.n_full - it.kb0, 0), it.n_total);
+  }
+  return nf * kFullCost + (it.n_total - nf) * kPartialCost;
+}
+
+int64_t item_cost(const WorkItem& it, const uint32_t* kblocks) {
+  return block_cost(it, kblocks) + (it.part >= 0 ? kPartOverhead : kItemOverhead);
+}
+
+// Longest processing time first; items are sorted by decreasing cost. Returns the owner of
 // every item and the makespan.
-int64_t lpt(const std::vector<WorkItem>& items, int32_t g, std::vector<int32_t>* owner) {
+int64_t lpt(const std::vector<WorkItem>& items, int32_t g, std::vector<int32_t>* owner, const uint32_t* kblocks) {
   using Load = std::pair<int64_t, int32_t>;  // (load, cta)
   std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
   for (int32_t c = 0; c < g; ++c) heap.push({0, c});
@@ -279,7 +301,7 @@ int64_t lpt(const std::vector<WorkItem>& items, int32_t g, std::vector<int32_t>*
     Load l = heap.top();
     heap.pop();
     (*owner)[i] = l.second;
-    l.first += item_cost(items[i]);
+    l.first += item_cost(items[i], kblocks);
     makespan = std::max(makespan, l.first);
     heap.push(l);
   }
@@ -291,17 +313,16 @@ int64_t lpt(const std::vector<WorkItem>& items, int32_t g, std::vector<int32_t>*
 // they can be split (prefix form, two or more key blocks), and the key blocks of those items
 // are handed out in parts, each part to the least-loaded CTA as much as fits under the
 // target (at least kMinPartBlocks). An item that ends up in one part stays whole.
-constexpr int64_t kPartOverhead = 3;  // an extra item's Q load, pipeline fill and epilogue
-constexpr int32_t kMinPartBlocks = 2;
 int64_t tail_split(const std::vector<WorkItem>& items, int32_t g, const std::vector<int32_t>& owner,
-                   std::vector<std::vector<WorkItem>>* lists, std::vector<WorkItem>* splits) {
+                   std::vector<std::vector<WorkItem>>* lists, std::vector<WorkItem>* splits,
+                   const uint32_t* kblocks) {
   lists->assign(static_cast<size_t>(g), {});
   std::vector<int64_t> load(static_cast<size_t>(g), 0);
   int64_t total = 0;
   for (size_t i = 0; i < items.size(); ++i) {
     (*lists)[static_cast<size_t>(owner[i])].push_back(items[i]);
-    load[static_cast<size_t>(owner[i])] += item_cost(items[i]);
-    total += item_cost(items[i]);
+    load[static_cast<size_t>(owner[i])] += item_cost(items[i], kblocks);
+    total += item_cost(items[i], kblocks);
   }
   const int64_t target = (total + g - 1) / g + kPartOverhead;
   std::vector<WorkItem> given;
@@ -310,7 +331,7 @@ int64_t tail_split(const std::vector<WorkItem>& items, int32_t g, const std::vec
     while (load[static_cast<size_t>(c)] > target && l.size() > 1) {
       const WorkItem& it = l.back();
       if (it.list_off >= 0 || it.part >= 0 || it.n_total < 2 * kMinPartBlocks) break;
-      load[static_cast<size_t>(c)] -= item_cost(it);
+      load[static_cast<size_t>(c)] -= item_cost(it, kblocks);
       given.push_back(it);
       l.pop_back();
     }
@@ -327,7 +348,7 @@ int64_t tail_split(const std::vector<WorkItem>& items, int32_t g, const std::vec
     while (remaining > 0) {
       Load l = heap.top();
       heap.pop();
-      int64_t k = std::max<int64_t>(kMinPartBlocks, target - l.first - kPartOverhead);
+      int64_t k = std::max<int64_t>(kMinPartBlocks, (target - l.first - kPartOverhead) / kFullCost);
       k = std::min<int64_t>(k, remaining);
       if (remaining - k > 0 && remaining - k < kMinPartBlocks) k = remaining;  // no tiny tail
       WorkItem part = it;
@@ -337,7 +358,7 @@ int64_t tail_split(const std::vector<WorkItem>& items, int32_t g, const std::vec
       auto& dst = (*lists)[static_cast<size_t>(l.second)];
       placed.emplace_back(l.second, dst.size());
       dst.push_back(part);
-      l.first += k + kPartOverhead;
+      l.first += item_cost(part, kblocks);
       heap.push(l);
       remaining -= static_cast<int32_t>(k);
       kb += static_cast<int32_t>(k);
@@ -366,6 +387,8 @@ int64_t tail_split(const std::vector<WorkItem>& items, int32_t g, const std::vec
 }
 
 }  // namespace
+
+int64_t planned_cost(const WorkItem& it, const uint32_t* kblocks) { return item_cost(it, kblocks); }
 
 void assign_ctas(Plan* plan, int32_t ctas, bool allow_split, bool force_split) {
   plan->splits.clear();
@@ -397,6 +420,9 @@ void assign_ctas(Plan* plan, int32_t ctas, bool allow_split, bool force_split) {
                      [](const WorkItem& x, const WorkItem& y) { return x.n_total > y.n_total; });
     plan->items.swap(halves);
   }
+  const uint32_t* kb = plan->kblocks.data();
+  std::stable_sort(plan->items.begin(), plan->items.end(),
+                   [kb](const WorkItem& x, const WorkItem& y) { return item_cost(x, kb) > item_cost(y, kb); });
   const int32_t n = static_cast<int32_t>(plan->items.size());
   const int32_t g = std::max(1, std::min(ctas, n));
   plan->grid = n ? g : 0;
@@ -404,13 +430,13 @@ void assign_ctas(Plan* plan, int32_t ctas, bool allow_split, bool force_split) {
   plan->makespan = 0;
   if (!n) return;
   std::vector<int32_t> owner;
-  const int64_t lpt_span = lpt(plan->items, g, &owner);
+  const int64_t lpt_span = lpt(plan->items, g, &owner, kb);
   std::vector<std::vector<WorkItem>> lists;
   std::vector<WorkItem> splits;
   int64_t span = lpt_span;
   bool use_split = false;
   if (allow_split && !force_split && g > 1) {
-    span = tail_split(plan->items, g, owner, &lists, &splits);
+    span = tail_split(plan->items, g, owner, &lists, &splits, kb);
     use_split = !splits.empty() && span + kSplitPenalty < lpt_span;
   }
   if (!use_split) {  // the longest-first lists, each CTA keeping the longest-first order

@@ -96,20 +96,30 @@ hgx_status check_first_rows(int32_t batch, const int32_t* cu_seqlens, const hgx_
                             const int32_t* cu_segs, const int32_t* first_rows, std::string* err);
 
 // Distributes plan->items over `ctas` persistent CTAs (longest-processing-time first: each
-// item, in decreasing cost, goes to the least loaded CTA; cost = key blocks + a per-item
-// overhead), reorders the items so that every CTA's list is contiguous, and sets grid,
+// item, in decreasing cost, goes to the least loaded CTA; cost = planned_cost: fully visible
+// key blocks, the dearer blocks that run the mask compare and a per-item overhead), reorders
+// the items so that every CTA's list is contiguous, and sets grid,
 // cta_offsets and makespan. grid = min(ctas, number of items).
 //
 // With allow_split, a second schedule is tried: the CTAs loaded above the mean give back
 // their last (smallest) items, whose key blocks are handed out in parts to the least-loaded
 // CTAs (tail_split in planner.cpp). It replaces the first schedule when its makespan plus
 // kSplitPenalty is smaller.
-constexpr int64_t kItemOverhead = 2;   // loading Q and writing O: about two key blocks
-constexpr int64_t kSplitPenalty = 3;   // the combine launch, in key blocks
+// Costs are in tenths of a fully visible key block (planner.cpp: a PARTIAL block costs 13).
+constexpr int64_t kItemOverhead = 12;  // loading Q, filling the pipeline, writing O
+constexpr int64_t kSplitPenalty = 30;  // the combine launch
 // force_split (a test hook that exercises the split path on any input): every prefix-form
 // item of two or more key blocks is split into two halves, then all items are assigned
 // longest first.
 void assign_ctas(Plan* plan, int32_t ctas, bool allow_split = false, bool force_split = false);
+
+// Cost of a work item in the assignment (tenths of a fully visible key block): 10 per fully
+// visible block, 13 per block that runs the mask compare, plus kItemOverhead (or the larger
+// overhead of a part of a split item). kblocks: the plan's key-block lists, needed only for
+// list-form items (may be NULL otherwise).
+int64_t planned_cost(const WorkItem& it, const uint32_t* kblocks);
+// The largest planned_cost of a prefix-form item of at most max_blocks key blocks.
+constexpr int64_t planned_cost_bound(int64_t max_blocks) { return 13 * max_blocks + kItemOverhead; }
 
 // Tile classes of every (query block, key block) of every batch element in order (after
 // a successful build_plan with the same descriptor).

@@ -267,8 +267,8 @@ def _config_dict(w):
     )
     d = {"workload": w.name, "tokens": w.total_tokens, "batch": len(w.batches), "segments": segs,
          "heads": "32q/8kv", "head_dim": 128, "mrope": "[24,20,20] theta 5e6",
-         "l2": f"inputs larger than L2: a distinct {48 * 128 * 2 * w.total_tokens / 1e6:.0f} MB "
-               f"(q, k, v) input set per step",
+         "l2": f"a distinct {48 * 128 * 2 * w.total_tokens / 1e6:.0f} MB (q, k, v) input set per step, "
+               f"the sets rotating over far more memory than L2 holds: no step finds its inputs in L2",
          "parallelism": "replicas (one full workload per GPU)"}
     return d
 

@@ -646,7 +646,7 @@ def run_gpu_layer(args):
         "dtype": "bf16",
         "data": "synthetic (random-init projection weights)",
         "config": dict(_config_dict(w), layer_gflop_per_step=round(flops / 1e9, 3),
-                       l2=f"inputs larger than L2: a distinct {x_bytes / 1e6:.0f} MB x per step"),
+                       l2=f"a distinct {x_bytes / 1e6:.0f} MB x per step, the inputs rotating over far more memory than L2 holds"),
         "kernel_ms": {"qkv_projection": ms[0], "attention": ms[1], "out_projection": ms[2]},
         "roofline": dict(bound="tensor", kernel="attention_kernel", unit="TFLOP/s", peak=peak, traffic=None,
                          peak_source=f"{peak_src} bf16 dense (burst)", **roof(att_flops, ms[1])),

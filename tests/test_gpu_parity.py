@@ -104,6 +104,29 @@ def test_prologue_matches_oracle(hgx, case):
         assert bool((pad == 7.0).all())
 
 
+def test_prologue_large_positions(hgx):
+    """Positions around and beyond 2^24, positive and negative: below 2^24 the kernel reduces
+    the angle in fp32 (position times a two-float split of inv_freq / 2 pi), from 2^24 on it
+    takes the fp64 sincos; both must match the fp64 oracle within bf16 rounding. Rows 0-15
+    straddle 2^24 by a few units, 16-31 reach 2^30, 32-47 go down to -2^30, and the three
+    axes of a row differ."""
+    H, a = hgx
+    w = W.custom("big_pos", [[(48, 0)]], seed=23)
+    t = W.tensors(w)
+    d = {n: x.cuda() for n, x in t.items()}
+    rng = np.random.default_rng(23)
+    pos = np.empty((48, 3), dtype=np.int64)
+    pos[:16] = (1 << 24) + rng.integers(-8, 8, size=(16, 3))
+    pos[16:32] = rng.integers(1 << 20, 1 << 30, size=(16, 3))
+    pos[32:48] = -rng.integers(1 << 20, 1 << 30, size=(16, 3))
+    pos = pos.astype(np.int32)
+    a.prologue(d["q"], d["k"], torch.from_numpy(pos).cuda(), d["wq"], d["wk"])
+    assert a.sync_status() == H.HGX_OK
+    qr, kr = O.prologue(t["q"], t["k"], pos, t["wq"], t["wk"])
+    np.testing.assert_allclose(d["q"].float().cpu().numpy(), qr, rtol=2.0 ** -8, atol=1e-5)
+    np.testing.assert_allclose(d["k"].float().cpu().numpy(), kr, rtol=2.0 ** -8, atol=1e-5)
+
+
 @pytest.mark.parametrize("layout", [1, 2])
 def test_prologue_2d_rope_layouts(hgx, layout):
     """HunyuanImage 3.0 Generalized 2D RoPE, both readings (x = w column, y = h column), on

@@ -72,6 +72,33 @@ def test_qkv_projection_with_fused_norm_and_rotation(hgx, cfg):
         np.testing.assert_allclose(got.float().cpu().numpy(), ref, rtol=2.0 ** -8, atol=2e-3)
 
 
+def test_qkv_projection_at_large_positions(hgx):
+    """The projection's (cos, sin) table (fp64 angles per token and frequency) at positions
+    around and beyond 2^24 and down to -2^30, against the oracle's rotation."""
+    H, a = hgx
+    w = W.config(0)
+    lt = W.layer_tensors(w)
+    d = {n: t.cuda() for n, t in lt.items()}
+    T = w.total_tokens
+    rng = np.random.default_rng(29)
+    pos = np.empty((T, 3), dtype=np.int64)
+    pos[: T // 3] = (1 << 24) + rng.integers(-8, 8, size=(T // 3, 3))
+    pos[T // 3: 2 * T // 3] = rng.integers(1 << 20, 1 << 30, size=(2 * T // 3 - T // 3, 3))
+    pos[2 * T // 3:] = -rng.integers(1 << 20, 1 << 30, size=(T - 2 * T // 3, 3))
+    pos = pos.astype(np.int32)
+    q = torch.empty(T, 32, 128, dtype=torch.bfloat16, device="cuda")
+    k = torch.empty(T, 8, 128, dtype=torch.bfloat16, device="cuda")
+    v = torch.empty(T, 8, 128, dtype=torch.bfloat16, device="cuda")
+    a.qkv_projection(d["x"], d["w_qkv"], q, k, v, torch.from_numpy(pos).cuda(), d["wq"], d["wk"])
+    assert a.sync_status() == H.HGX_OK
+    q_r, k_r, _ = O.qkv_projection(lt["x"], lt["w_qkv"])
+    phi = O.mrope_angles(pos, 5e6, 128, (24, 20, 20))
+    qp = O.rope_rotate_half(O.rms_norm(q_r, O.bf16_to_f64(lt["wq"]), 1e-6), phi)
+    kp = O.rope_rotate_half(O.rms_norm(k_r, O.bf16_to_f64(lt["wk"]), 1e-6), phi)
+    for got, ref in ((q, qp), (k, kp)):
+        np.testing.assert_allclose(got.float().cpu().numpy(), ref, rtol=2.0 ** -8, atol=2e-3)
+
+
 def _layer(hgx, w):
     H, a = hgx
     lt = W.layer_tensors(w)

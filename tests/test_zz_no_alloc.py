@@ -113,6 +113,26 @@ def test_noalloc_matches_forward_on_two_calls_in_a_row(lib):
         _within(got[rows], _oracle_rows(w, rows), w.name + " vs oracle")
 
 
+def test_noalloc_at_its_size_limit(lib):
+    """16 384 packed tokens in 64 batch elements (the most the fixed scratch takes), ragged
+    lengths of 257 and 193 tokens (every element ends one token into a query block), causal
+    text then a full_in_segment image: against hgx_attn_forward, and against the oracle on one
+    row of every 64-token query block plus each element's first and last row."""
+    B = lib
+    lens = [257] * 63 + [16384 - 63 * 257]
+    w = W.custom("noalloc_max", [[(17, 0), (n - 17, 2)] for n in lens], seed=31)
+    assert w.total_tokens == 16384 and len(w.batches) == 64
+    got = _noalloc(B, w).float().cpu().numpy()
+    ref = _regular(B, w).float().cpu().numpy()
+    _within(got, ref, "limit vs hgx_attn_forward")
+    cu = W.cu_seqlens(w)
+    rng = np.random.default_rng(31)
+    rows = {int(rng.integers(r0, min(w.total_tokens, r0 + 64))) for r0 in range(0, w.total_tokens, 64)}
+    rows |= {int(c) for c in cu[:-1]} | {int(c) - 1 for c in cu[1:]}
+    rows = sorted(rows)
+    _within(got[rows], _oracle_rows(w, rows), "limit vs oracle")
+
+
 def test_noalloc_rejects_sizes_beyond_its_limit(lib):
     B = lib
     cfg = B.Attention.default_config()

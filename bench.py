@@ -41,6 +41,9 @@ sys.path.insert(0, ROOT)
 import workloads as W  # noqa: E402
 
 FLOP_PER_PAIR = 4 * W.HEAD_DIM * W.NUM_Q_HEADS
+# the tensor core of one SM: a dense bf16 MMA of 128 x 128 x 16 (524 288 FLOP) every 64 cycles
+# (2.25 PFLOP/s nominal = 148 SMs x 8192 x ~1.86 GHz)
+DENSE_BF16_FLOP_PER_SM_CYCLE = 8192
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 SET_BUDGET_BYTES = 24e9
 
@@ -279,6 +282,16 @@ PER_WORKLOAD = ("hidream_tiny_321", "hidream_t2i_1024_cfg", "hidream_t2i_2048_cf
 L2_FLUSH_BYTES = 256 << 20  # twice the 126 MB L2
 
 
+def _kernel_clock_entry(cycles, span_ns, mhz, flops, n_sm, which):
+    """The attention kernel's own clock stamps (clock64 and %globaltimer at every CTA's start
+    and end): cycles of the slowest CTA, the effective SM clock (median over CTAs), and the
+    algorithmic FLOPs over what the tensor cores could do in those cycles."""
+    return {"launch": which, "attention_cycles": cycles, "attention_span_us": span_ns / 1e3,
+            "effective_sm_mhz": round(mhz, 1),
+            "tensor_frac_of_cycles": flops / (cycles * n_sm * DENSE_BF16_FLOP_PER_SM_CYCLE),
+            "tensor_rate": f"{DENSE_BF16_FLOP_PER_SM_CYCLE} dense bf16 FLOP per SM per cycle x {n_sm} SMs"}
+
+
 def per_workload_timings(H, a, peaks, iters=10, names=PER_WORKLOAD):
     """Event-timed prologue and attention launches of every workload, each launch preceded by
     an L2 flush outside the timed launch (a write of a buffer twice the size of L2, then a
@@ -326,12 +339,16 @@ def per_workload_timings(H, a, peaks, iters=10, names=PER_WORKLOAD):
                 att.append(ev[2].elapsed_time(ev[3]))
         if a.sync_status(stream) != H.HGX_OK:
             raise RuntimeError(a.last_error())
+        cyc, span_ns, mhz = a.kernel_clock(stream)  # the last of these launches
+        n_sm = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
         att_ms, pro_ms = statistics.median(att), statistics.median(pro)
         tf = flops / (att_ms * 1e-3) / 1e12
         gbs = 80 * 128 * 2 * T / (pro_ms * 1e-3) / 1e9
         res[name] = {"tokens": T, "unmasked_gflop": round(flops / 1e9, 3),
                      "attention_ms": att_ms, "attention_tflops": tf, "attention_frac": tf / peaks["bf16_tflops"],
                      "prologue_ms": pro_ms, "prologue_gbs": gbs, "prologue_frac": gbs / peaks["hbm_gbs"],
+                     "attention_cycles": cyc, "effective_sm_mhz": round(mhz, 1),
+                     "tensor_frac_of_cycles": flops / (cyc * n_sm * DENSE_BF16_FLOP_PER_SM_CYCLE),
                      "oracle_tflops": None}
         del d, pristine, v, out
     return res
@@ -414,6 +431,9 @@ def run_gpu(args):
     if a.sync_status(stream) != H.HGX_OK:
         raise RuntimeError(a.last_error())
     elapsed_ms = start.elapsed_time(stop)
+    # the last timed step's attention launch, from the kernel's own clock stamps
+    att_cycles, att_span_ns, att_mhz = a.kernel_clock(stream)
+    n_sm = torch.cuda.get_device_properties(local).multi_processor_count
     _log(f"timed {args.steps} steps: {elapsed_ms / args.steps:.3f} ms per step")
     pro_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
     att_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
@@ -530,6 +550,8 @@ def run_gpu(args):
         "gpu_launches": (1 + (sum(1 for b in range(len(w.batches)) if first_rows[b] < w.lengths[b])
                               if first_rows else 1) + (1 if _has_splits(w, first_rows) else 0)) * args.steps,
         "clocks": clk.summary(),
+        "kernel_clock": _kernel_clock_entry(att_cycles, att_span_ns, att_mhz, flops, n_sm,
+                                            "the last timed step's attention launch"),
     }
     del sets
     if not args.no_per_workload and not first_rows:

@@ -263,6 +263,18 @@ hgx_status hgx_attn_schedule(int32_t batch, const int32_t* cu_seqlens_host,
  * stream reports an error, HGX_OK otherwise. */
 hgx_status hgx_attn_sync_status(hgx_attn_handle* h, void* stream);
 
+/* Clock of the last attention launch made through h (hgx_attn_forward, _forward_from,
+ * _attention or _layer_forward); the pages have no counterpart, this is measurement. Every
+ * persistent CTA of the attention kernel stamps the SM's cycle counter (clock64) and the
+ * global nanosecond timer at its start and at its end into a small device buffer that the
+ * handle owns. This call synchronizes `stream`, copies the stamps and returns: *cycles =
+ * the largest CTA's cycle count, *ns = the largest CTA's span in nanoseconds, *sm_mhz =
+ * the median over CTAs of cycles / ns (the effective SM clock, which under the power cap
+ * can sit well below the clock NVML reports). HGX_ERR_INVALID_ARG if a pointer is NULL or
+ * no attention kernel has run on this handle; the call does not clear the error word. */
+hgx_status hgx_attn_kernel_clock(hgx_attn_handle* h, void* stream, uint64_t* cycles, uint64_t* ns,
+                                 double* sm_mhz);
+
 /* Debug flags for hgx_attn_set_debug. */
 #define HGX_DEBUG_CHECKED 1u    /* every device call ends with hgx_attn_sync_status */
 #define HGX_DEBUG_STALL_TEST 2u /* attention: one softmax warpgroup first waits on a barrier

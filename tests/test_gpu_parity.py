@@ -530,3 +530,35 @@ def test_split_items_and_combine_elementwise(hgx, case):
         _compare(out.float().cpu().numpy(), ref, f"split {w.name}")
     finally:
         a.close()
+
+
+def test_kernel_clock_stamps_of_the_last_attention_launch(hgx):
+    """hgx_attn_kernel_clock: refused before any attention launch; afterwards the slowest
+    CTA's cycles and span, and an effective SM clock that agrees with them and with the
+    event-timed launch."""
+    H, _ = hgx
+    a = H.Attention()
+    try:
+        with pytest.raises(H.HgxError):
+            a.kernel_clock()
+        w = W.CONFIG_BY_NAME["hidream_t2i_1024_cfg"]
+        _, d = _device_inputs(w)
+        cu, segs, cu_segs = _desc(w)
+        a.prologue(d["q"], d["k"], d["pos"], d["wq"], d["wk"])
+        out = _nan_like(d["q"])
+        stream = torch.cuda.current_stream()
+        for _ in range(3):  # the plan is uploaded by the first call
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            a.attention(d["q"], d["k"], d["v"], out, cu, segs, cu_segs)
+            e1.record(stream)
+        cyc, ns, mhz = a.kernel_clock()
+        assert a.sync_status() == H.HGX_OK
+        assert bool(torch.isfinite(out).all())
+        launch_ms = e0.elapsed_time(e1)
+        assert cyc > 0 and ns > 0
+        assert 300.0 < mhz < 2500.0, mhz
+        assert ns * 1e-6 <= launch_ms * 1.02 + 0.005, (ns, launch_ms)  # inside the launch
+        assert abs(cyc / (ns * 1e-3) / mhz - 1.0) < 0.1, (cyc, ns, mhz)
+    finally:
+        a.close()

@@ -63,6 +63,8 @@ _SIGS = {
     "hgx_attn_schedule": (ctypes.c_int, [ctypes.c_int32] + [ctypes.c_void_p] * 3 + [ctypes.c_int32, ctypes.c_int32,
                           ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "hgx_attn_sync_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
+    "hgx_attn_kernel_clock": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint64),
+                                             ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_double)]),
     "hgx_attn_set_debug": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_uint32, ctypes.c_uint64]),
 }
 
@@ -324,6 +326,14 @@ class Attention:
     def sync_status(self, stream=None) -> int:
         """Synchronizes the stream; returns the status code (HGX_ERR_TIMEOUT after a wait ran out)."""
         return lib().hgx_attn_sync_status(self._h, _stream_ptr(stream))
+
+    def kernel_clock(self, stream=None):
+        """(cycles of the slowest CTA, its span in ns, median effective SM clock in MHz) of the
+        last attention launch on this handle; synchronizes the stream."""
+        cyc, ns, mhz = ctypes.c_uint64(), ctypes.c_uint64(), ctypes.c_double()
+        self._check(lib().hgx_attn_kernel_clock(self._h, _stream_ptr(stream), ctypes.byref(cyc), ctypes.byref(ns),
+                                                ctypes.byref(mhz)), "hgx_attn_kernel_clock")
+        return int(cyc.value), int(ns.value), float(mhz.value)
 
     def set_debug(self, flags: int, wait_limit_ns: int = 0):
         self._check(lib().hgx_attn_set_debug(self._h, flags, wait_limit_ns), "hgx_attn_set_debug")

@@ -7,6 +7,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
@@ -61,6 +62,9 @@ struct hgx_attn_handle {
   void* d_rope_cs = nullptr;
   size_t rope_cs_cap = 0;
   uint32_t* d_err = nullptr;
+  // per-CTA clock64 / %globaltimer stamps of the last attention launch ([num_sms][4])
+  uint64_t* d_stamps = nullptr;
+  int stamps_grid = 0;
   // pinned staging for the plan upload, reused once the previous upload has completed
   uint8_t* h_stage = nullptr;
   size_t stage_cap = 0;
@@ -153,6 +157,8 @@ hgx_status ensure_device(hgx_attn_handle* h) {
   if (e != cudaSuccess) return fail(h, HGX_ERR_OOM, "cudaMalloc of the error word failed");
   e = cudaMemset(h->d_err, 0, sizeof(uint32_t));
   if (e != cudaSuccess) return cuda_fail(h, e, "cudaMemset");
+  e = cudaMalloc(&h->d_stamps, static_cast<size_t>(h->num_sms) * 4 * sizeof(uint64_t));
+  if (e != cudaSuccess) return fail(h, HGX_ERR_OOM, "cudaMalloc of the clock stamps failed");
   e = cudaEventCreateWithFlags(&h->stage_done, cudaEventDisableTiming);
   if (e != cudaSuccess) return cuda_fail(h, e, "cudaEventCreate");
   h->device = dev;
@@ -330,8 +336,10 @@ hgx_status run_attention(hgx_attn_handle* h, cudaStream_t stream, const void* q,
   p.flags = h->flags;
   p.err = h->d_err;
   p.wait_limit_ns = h->wait_limit_ns;
+  p.stamps = h->d_stamps;
   cudaError_t e = hgx::launch_attention(stream, mq, mk, mv, mo, p, h->plan.grid);
   if (e != cudaSuccess) return cuda_fail(h, e, "attention launch");
+  h->stamps_grid = h->plan.grid;
   if (slots) {
     e = hgx::launch_combine(stream, h->d_splits, static_cast<int32_t>(h->plan.splits.size()), p.partial_o,
                             p.partial_ml, out);
@@ -465,6 +473,7 @@ void hgx_attn_destroy(hgx_attn_handle* h) {
   if (h->d_partial) cudaFree(h->d_partial);
   if (h->d_rope_cs) cudaFree(h->d_rope_cs);
   if (h->d_err) cudaFree(h->d_err);
+  if (h->d_stamps) cudaFree(h->d_stamps);
   if (h->h_stage) cudaFreeHost(h->h_stage);
   if (h->stage_done) cudaEventDestroy(h->stage_done);
   delete h;
@@ -729,6 +738,32 @@ hgx_status hgx_attn_sync_status(hgx_attn_handle* h, void* stream) {
     std::snprintf(buf, sizeof(buf), "a bounded device wait ran out (error word 0x%08x)", word);
     return fail(h, HGX_ERR_TIMEOUT, buf);
   }
+  return HGX_OK;
+}
+
+hgx_status hgx_attn_kernel_clock(hgx_attn_handle* h, void* stream, uint64_t* cycles, uint64_t* ns,
+                                 double* sm_mhz) {
+  if (!h || !cycles || !ns || !sm_mhz) return HGX_ERR_INVALID_ARG;
+  if (h->stamps_grid <= 0) return fail(h, HGX_ERR_INVALID_ARG, "no attention launch on this handle yet");
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(h, e, "cudaStreamSynchronize");
+  std::vector<uint64_t> st(static_cast<size_t>(h->stamps_grid) * 4);
+  e = cudaMemcpy(st.data(), h->d_stamps, st.size() * sizeof(uint64_t), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(h, e, "cudaMemcpy (clock stamps)");
+  uint64_t cmax = 0, nmax = 0;
+  std::vector<double> mhz;
+  for (int c = 0; c < h->stamps_grid; ++c) {
+    const uint64_t* s = &st[4 * static_cast<size_t>(c)];
+    if (s[2] < s[0] || s[3] <= s[1]) return fail(h, HGX_ERR_CUDA, "clock stamps out of order");
+    const uint64_t dc = s[2] - s[0], dn = s[3] - s[1];
+    cmax = std::max(cmax, dc);
+    nmax = std::max(nmax, dn);
+    mhz.push_back(1e3 * static_cast<double>(dc) / static_cast<double>(dn));
+  }
+  std::nth_element(mhz.begin(), mhz.begin() + mhz.size() / 2, mhz.end());
+  *cycles = cmax;
+  *ns = nmax;
+  *sm_mhz = mhz[mhz.size() / 2];
   return HGX_OK;
 }
 

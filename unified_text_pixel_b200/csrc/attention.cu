@@ -266,6 +266,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  if (p.stamps && threadIdx.x == 0) {
+    p.stamps[4 * blockIdx.x] = clock64();
+    p.stamps[4 * blockIdx.x + 1] = globaltimer_ns();
+  }
 
   // Registers (one warp per row): launched at 168 per thread (384 x 168 = 64512). The
   // producer/MMA warpgroup hands registers to the two softmax warpgroups: 128 x 120 +
@@ -441,6 +445,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) {
       tc_fence_after();
       tmem_dealloc(tmem, kTmemCols);
+    }
+    if (p.stamps && threadIdx.x == 0) {  // every role of the CTA has passed the barrier
+      p.stamps[4 * blockIdx.x + 2] = clock64();
+      p.stamps[4 * blockIdx.x + 3] = globaltimer_ns();
     }
   } else {
     if constexpr (kRegsLow != kRegsHigh) regs_increase<kRegsHigh>();

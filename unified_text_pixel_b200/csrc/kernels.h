@@ -40,6 +40,8 @@ struct AttnParams {
   uint32_t flags;          // HGX_DEBUG_* bits
   uint32_t* err;           // device error word (sticky until read)
   uint64_t wait_limit_ns;  // bound of every wait
+  uint64_t* stamps;        // NULL, or [grid][4]: per CTA clock64 and %globaltimer at its start
+                           // and at its end (the effective SM clock of the launch)
 };
 
 // Merges the partial results of every split item into out (bf16):

@@ -238,6 +238,21 @@ def test_set_debug_rejects_unknown_flags():
     a.close()
 
 
+def test_kernel_clock_refuses_before_any_launch():
+    """hgx_attn_kernel_clock needs a handle that has launched the attention kernel; the
+    refusals come before any CUDA call."""
+    L = B.lib()
+    c, n, m = ctypes.c_uint64(), ctypes.c_uint64(), ctypes.c_double()
+    assert L.hgx_attn_kernel_clock(None, None, ctypes.byref(c), ctypes.byref(n), ctypes.byref(m)) == B.HGX_ERR_INVALID_ARG
+    a = B.Attention()
+    assert L.hgx_attn_kernel_clock(a.handle, None, None, ctypes.byref(n), ctypes.byref(m)) == B.HGX_ERR_INVALID_ARG
+    with pytest.raises(B.HgxError) as e:
+        a.kernel_clock(stream=0)  # the legacy default stream: no torch stream needed here
+    assert e.value.status == B.HGX_ERR_INVALID_ARG
+    assert "no attention launch" in a.last_error()
+    a.close()
+
+
 def test_library_exports_every_declared_symbol():
     with open(os.path.join(ROOT, "include", "hgx_attn.h")) as f:
         text = f.read()

@@ -530,6 +530,10 @@ def run_gpu(args):
             "traffic": traffic,
             "peak_source": f"{peak_src} bf16 dense (burst; the kernel is timed inside a short step)",
             "algorithmic_flop_per_launch": flops,
+            # context, not the headline: inside the timed loop the kernel runs under the power
+            # cap (see kernel_clock), as the sustained GEMM figure does
+            "peak_sustained": peaks["bf16_tflops_sustained"],
+            "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
         },
         "prologue_roofline": {
             "bound": "hbm",

@@ -153,14 +153,38 @@ hgx_status ensure_device(hgx_attn_handle* h) {
     return fail(h, HGX_ERR_UNSUPPORTED, "this library is built for sm_100a (B200) only");
   e = cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return cuda_fail(h, e, "cudaDeviceGetAttribute");
+  // on failure, release what this call allocated, so that the handle stays unbound and
+  // holds nothing of this device
+  auto undo = [h]() {
+    if (h->d_err) cudaFree(h->d_err);
+    if (h->d_stamps) cudaFree(h->d_stamps);
+    if (h->stage_done) cudaEventDestroy(h->stage_done);
+    h->d_err = nullptr;
+    h->d_stamps = nullptr;
+    h->stage_done = nullptr;
+  };
   e = cudaMalloc(&h->d_err, sizeof(uint32_t));
-  if (e != cudaSuccess) return fail(h, HGX_ERR_OOM, "cudaMalloc of the error word failed");
+  if (e != cudaSuccess) {
+    h->d_err = nullptr;
+    return fail(h, HGX_ERR_OOM, "cudaMalloc of the error word failed");
+  }
   e = cudaMemset(h->d_err, 0, sizeof(uint32_t));
-  if (e != cudaSuccess) return cuda_fail(h, e, "cudaMemset");
+  if (e != cudaSuccess) {
+    undo();
+    return cuda_fail(h, e, "cudaMemset");
+  }
   e = cudaMalloc(&h->d_stamps, static_cast<size_t>(h->num_sms) * 4 * sizeof(uint64_t));
-  if (e != cudaSuccess) return fail(h, HGX_ERR_OOM, "cudaMalloc of the clock stamps failed");
+  if (e != cudaSuccess) {
+    h->d_stamps = nullptr;
+    undo();
+    return fail(h, HGX_ERR_OOM, "cudaMalloc of the clock stamps failed");
+  }
   e = cudaEventCreateWithFlags(&h->stage_done, cudaEventDisableTiming);
-  if (e != cudaSuccess) return cuda_fail(h, e, "cudaEventCreate");
+  if (e != cudaSuccess) {
+    h->stage_done = nullptr;
+    undo();
+    return cuda_fail(h, e, "cudaEventCreate");
+  }
   h->device = dev;
   return HGX_OK;
 }

@@ -178,6 +178,21 @@ def test_forward_gen_image_holes_elementwise(hgx, seed):
     _compare(out.float().cpu().numpy(), ref, w.name)
 
 
+@pytest.mark.parametrize("seed", range(8))
+def test_forward_larger_mixed_layouts_elementwise(hgx, seed):
+    """All four segment kinds (Gen Image holes included) in up to three elements of up to
+    1600 tokens, empty elements allowed: several items per CTA of different lengths, so the
+    planner's longest-first lists and tail splits (with their combine launch) take part;
+    element by element against the oracle's dense mask."""
+    w = W.random_workload(300 + seed, max_batch=3, max_len=1600, allow_empty=True, kinds=(0, 1, 2, 3))
+    if w.total_tokens == 0:
+        pytest.skip("empty draw")
+    t, _ = _device_inputs(w)
+    out, _ = _run(hgx, w)
+    ref, _, _ = _oracle_full(w, t)
+    _compare(out.float().cpu().numpy(), ref, w.name)
+
+
 def test_forward_multigen_full_size_sampled_rows(hgx):
     w = W.CONFIG_BY_NAME["hunyuan_multigen_9088"]
     t, _ = _device_inputs(w)

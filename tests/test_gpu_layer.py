@@ -132,6 +132,20 @@ def test_layer_forward_elementwise(hgx, cfg):
     _check(y.float().cpu().numpy(), y_r, "y")
 
 
+@pytest.mark.parametrize("seed", range(3))
+def test_layer_forward_random_layouts_elementwise(hgx, seed):
+    """The whole layer on random packed layouts (all four segment kinds, ragged elements,
+    Gen Image holes): row counts that end inside a 128-row GEMM tile, and batch elements
+    that start inside one."""
+    w = W.random_workload(500 + seed, max_batch=3, max_len=900, kinds=(0, 1, 2, 3))
+    lt, y, att = _layer(hgx, w)
+    segs, cu_segs = W.flat_segments(w)
+    y_r, att_r, _, _, _ = O.layer_forward(lt["x"], lt["w_qkv"], lt["w_o"], W.positions(w), lt["wq"], lt["wk"],
+                                          W.cu_seqlens(w), segs, cu_segs)
+    _check(att.float().cpu().numpy(), att_r, w.name + " attention")
+    _check(y.float().cpu().numpy(), y_r, w.name + " y")
+
+
 def test_layer_forward_full_size_sampled_rows(hgx):
     """The edit step's layer (8449 tokens): att and y are NaN-filled before the call and
     must come back finite everywhere; one random row of every 64-token query block (every

@@ -704,12 +704,18 @@ def _recorded_traffic(name):
 
 
 def _kernel_sha():
+    """Hash of the attention kernel's sources with comments and blank space removed, so that
+    a change of wording alone keeps the recorded counters."""
     import hashlib
+    import re
 
     hsh = hashlib.sha256()
     for f in ("attention.cu", "sm100.cuh", "kernels.h", "planner.h", "exp2_poly.h", "waits.cuh"):
-        with open(os.path.join(ROOT, "unified_text_pixel_b200", "csrc", f), "rb") as fh:
-            hsh.update(fh.read())
+        with open(os.path.join(ROOT, "unified_text_pixel_b200", "csrc", f), encoding="utf-8") as fh:
+            src = fh.read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", " ", src)
+        hsh.update(" ".join(src.split()).encode())
     return hsh.hexdigest()[:16]
 
 

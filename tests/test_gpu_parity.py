@@ -193,6 +193,22 @@ def test_forward_larger_mixed_layouts_elementwise(hgx, seed):
     _compare(out.float().cpu().numpy(), ref, w.name)
 
 
+def test_forward_many_tiny_elements_elementwise(hgx):
+    """300 packed elements of 1 to 39 tokens in one to three segments of mixed kinds: hundreds
+    of short work items, each ending inside a key block, several per CTA; element by element
+    against the oracle."""
+    rng = np.random.default_rng(77)
+    batches = []
+    for _ in range(300):
+        n_seg = int(rng.integers(1, 4))
+        batches.append([(int(rng.integers(1, 14)), int(rng.choice([0, 1, 2, 3]))) for _ in range(n_seg)])
+    w = W.custom("tiny300", batches, seed=77)
+    t, _ = _device_inputs(w)
+    out, _ = _run(hgx, w)
+    ref, _, _ = _oracle_full(w, t)
+    _compare(out.float().cpu().numpy(), ref, w.name)
+
+
 def test_forward_multigen_full_size_sampled_rows(hgx):
     w = W.CONFIG_BY_NAME["hunyuan_multigen_9088"]
     t, _ = _device_inputs(w)
